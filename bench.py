@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward (tokens/s) through the libmoe C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+One step = one whole layer forward (router, top-k, dispatch, expert FFNs,
+combine, aux statistics: six kernel launches) over one batch of the workload,
+inputs resident in HBM.  A 256 MiB buffer (twice the L2) is written between
+steps, outside the timed events, so every step starts with a cold L2.  Each
+step is timed with CUDA events on the launching stream; the per-stage events
+(recorded by moe_forward_profiled between the launches) give the dominant
+kernel's duration for the roofline.  Under torchrun each rank runs its own
+independent batch (weak scaling, no collective on the data path); the time
+is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (numpy, float64) on the host cores
+on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s; grouped-FFN TFLOP/s & HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "llama4moe_t4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+FLUSH_BYTES = 256 << 20
+ORACLE_SAMPLE_TOKENS = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- oracle timing
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_step(wl, inp, tokens):
+    """One bounded sample of the workload on the CPU oracle: routing of all
+    tokens, expert FFNs and combine for `tokens`."""
+    from oracle import moe_oracle as O
+    r = O.route(wl, inp)
+    O.forward(wl, inp, routing=r, tokens=tokens)
+
+
+def time_oracle(wl, inp, steps=None, seconds=None, warmup=0):
+    import numpy as np
+    tokens = np.arange(min(ORACLE_SAMPLE_TOKENS, wl.T))
+    for _ in range(warmup):
+        oracle_step(wl, inp, tokens)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(wl, inp, tokens)
+        n += 1
+        el = time.perf_counter() - t0
+        if (steps is not None and n >= steps) or (seconds is not None and el >= seconds):
+            break
+    return {"value": n * len(tokens) / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle steps; each routes all T={wl.T} tokens and computes the expert FFNs and "
+                      f"combine (float64, numpy/BLAS) for {len(tokens)} of them; value = output tokens / second",
+            "seconds": round(el, 3)}
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_id: str):
+        self.proc = None
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", dev_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# --------------------------------------------------------------------------- native
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "mixture_experts_layer_37_b200", "csrc", "gemm_sm100.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(f"{kernel}@{workload}")
+    if not ent or ent.get("source_sha") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def run_native(a):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_layer_37_b200 as M
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    wl = W.WORKLOADS[a.workload]
+    cfg = M.MoEConfig.of(wl)
+    seed = wl.seed + 1000 * rank
+    inp = W.make_inputs(wl, seed=seed)
+
+    def dev(arr):
+        if arr.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(arr)).cuda()
+
+    weights = {n: dev(inp[n]) for n in ("w_router", "w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2") if n in inp}
+    if inp.get("router_bias") is not None:
+        weights["router_bias"] = dev(np.asarray(inp["router_bias"], dtype=np.float32))
+    x = dev(inp["x"])
+    layer = M.MoELayer(cfg, weights)
+    nl = M.moe_forward_launch_count(cfg)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def make_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    for _ in range(a.warmup):
+        flush.zero_()
+        layer.forward(x)
+    torch.cuda.synchronize()
+    layer.check()
+
+    steps = [make_events(nl + 1) for _ in range(a.steps)]
+    torch.cuda.synchronize()
+    dev_id = str(torch.cuda.get_device_properties(local).uuid) if hasattr(torch.cuda.get_device_properties(local), "uuid") else str(local)
+    if not dev_id.startswith("GPU-") and len(dev_id) > 8:
+        dev_id = "GPU-" + dev_id
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev_id)
+    time.sleep(0.2)
+    for i in range(a.steps):
+        flush.zero_()
+        M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, steps[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    layer.check()
+
+    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in steps])
+    step_ms = np.array([ev[0].elapsed_time(ev[nl]) for ev in steps])
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * wl.T * a.steps / (total_ms / 1e3)
+
+    # ---------------- roofline of the dominant kernel
+    R = int(layer.outputs["offsets"][-1].item())
+    names = ["router", "scan", "scatter", "gemm1", "gemm2", "combine"]
+    mean_stage = stage_ms.mean(axis=0)
+    pk, pk_src = peaks()
+    bpe = 2 if wl.dtype == "bf16" else 4
+    gemm1_flops = (4 if wl.act == "swiglu" else 2) * wl.d * wl.ffn * R
+    gemm2_flops = 2 * wl.d * wl.ffn * R
+    algo = {
+        "router": ("hbm", wl.T * wl.d * bpe + wl.d * wl.E * bpe + wl.T * wl.k * 8),
+        "scan": ("hbm", 0),
+        "scatter": ("hbm", 2 * R * wl.d * bpe + wl.T * wl.k * 4 * 3),
+        "gemm1": ("tensor", gemm1_flops),
+        "gemm2": ("tensor", gemm2_flops),
+        "combine": ("hbm", R * wl.d * bpe + wl.T * wl.d * bpe + wl.T * wl.k * 8),
+    }
+    dom = int(np.argmax(mean_stage))
+    dname = names[dom]
+    bound, work = algo[dname]
+    dur_s = mean_stage[dom] / 1e3
+    if bound == "tensor":
+        achieved = work / dur_s / 1e12
+        peak = pk["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = work / dur_s / 1e9
+        peak = pk["hbm_gbs"]
+        unit = "GB/s"
+    roofline = {"bound": bound, "kernel": f"grouped_gemm_kernel ({dname})" if bound == "tensor" else dname,
+                "achieved": round(achieved, 2), "peak": peak, "peak_source": f"{pk_src} ({'bf16 dense burst' if bound == 'tensor' else 'HBM copy'})",
+                "unit": unit, "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic(dname, a.workload) if bound == "tensor" else None}
+    stages = {}
+    for j, n in enumerate(names):
+        b, w = algo[n]
+        ent = {"ms": round(float(mean_stage[j]), 4)}
+        if b == "tensor":
+            ent["TFLOP/s"] = round(w / (mean_stage[j] / 1e3) / 1e12, 1)
+        elif w:
+            ent["GB/s"] = round(w / (mean_stage[j] / 1e3) / 1e9, 1)
+        stages[n] = ent
+
+    # ---------------- end to end through the host-buffer entry point
+    x_host = torch.from_numpy(np.ascontiguousarray(inp["x"]).view(np.int16)).view(torch.bfloat16).pin_memory() \
+        if wl.dtype == "bf16" else torch.from_numpy(inp["x"]).pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    l_host = torch.empty(1, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_ev = [make_events(2) for _ in range(a.steps)]
+    for _ in range(max(1, a.warmup // 2)):
+        flush.zero_()
+        M.moe_forward_hostio(cfg, weights, x_host, x_dev, layer.outputs, out_host, l_host, layer.ws)
+    torch.cuda.synchronize()
+    for i in range(a.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        M.moe_forward_hostio(cfg, weights, x_host, x_dev, layer.outputs, out_host, l_host, layer.ws)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = float(sum(ev[0].elapsed_time(ev[1]) for ev in e2e_ev))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    layer.check()
+    bx = wl.T * wl.d * bpe
+    e2e = {"value": round(world * wl.T * a.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+           "h2d_bytes_per_step": bx, "d2h_bytes_per_step": bx + 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = time_oracle(wl, inp, seconds=a.cpu_baseline_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, generated on host)",
+        "config": {"workload": a.workload, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
+                   "act": wl.act, "capacity_factor": wl.capacity_factor, "rows_dispatched": R,
+                   "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "256 MiB buffer written between steps, outside the timed events"},
+        "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * a.steps,
+        "clocks": clocks, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference(a):
+    import workloads as W
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[a.workload]
+    inp = W.make_inputs(wl)
+    res = time_oracle(wl, inp, steps=a.steps, warmup=a.warmup)
+    line = {"metric": METRIC, "value": round(res["value"], 3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(1e3 * res["seconds"] / a.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, generated on host)",
+            "config": {"workload": a.workload, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
+                       "act": wl.act, "capacity_factor": wl.capacity_factor},
+            "impl": "reference",
+            "cpu_baseline": {"kind": "oracle", "cores": res["cores"], "sample": res["sample"], "value": round(res["value"], 3),
+                             "unit": UNIT},
+            "e2e": {"value": round(res["value"], 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_native(a)
+
+
+if __name__ == "__main__":
+    main()

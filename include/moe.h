@@ -1,0 +1,229 @@
+/*
+ * moe.h -- C ABI of libmoe, the forward pass of a top-k routed
+ * Mixture-of-Experts FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (pages that define it, by title and section):
+ *   router        score = x . W_r, a bias-free linear router, then a softmax
+ *                 over all E experts ("MoE: gating, experts, load balancing,
+ *                 capacity factor" (dpshk.com/news/6005940) §2.1);
+ *   top-k         the k experts with the largest logits, their probabilities
+ *                 renormalised to sum to 1 ("Llama-MoE架构解析" (coreui.cn
+ *                 /article/2610641) §3.1; MoE-basics page §3.1);
+ *   capacity      cap = ceil(T*k/E * capacity_factor); assignments beyond
+ *                 an expert's cap are dropped in token order (MoE-basics §2.4);
+ *   dispatch      assignments sorted by expert into contiguous groups
+ *                 ("Hand-building a LLaMA4-MoE" (dpshk.com/news/5809432) §2.4);
+ *   experts       SwiGLU (MoE-basics §2.2; Llama-MoE §2.1) or a two-matrix
+ *                 FFN with bias and GELU over one flattened [E, d, ffn] weight
+ *                 pool ("How to Loop MoE: Flatten the Experts, Untie the
+ *                 Attention" (discosf.com/news/5228035) §2.1; MoE-basics §3.1);
+ *   combine       out[t] = sum_j w[t,j] * expert_j(x[t]) (LLaMA4-MoE §2.4);
+ *   load balance  f_e, p_e and L_aux = alpha * E * sum_e f_e p_e
+ *                 (MoE-basics §2.3; LLaMA4-MoE §3.2).
+ *
+ * Conventions (all entry points):
+ *   - Every tensor pointer is DEVICE memory owned by the caller, row-major,
+ *     contiguous, 16-byte aligned, unless the comment says HOST.  The
+ *     library never allocates or frees memory and never synchronises, except
+ *     in moe_check_device_status (which synchronises the given stream).
+ *   - "act" tensors (x, x_perm, h, y_perm, out and the weights) have the
+ *     config's dtype: float32 (MOE_DT_F32) or bfloat16 (MOE_DT_BF16).
+ *     Router logits, probabilities, top-k weights, f, p and L_aux are float32;
+ *     indices and counts are int32.  The router logit bias is float32.
+ *   - Arguments are validated on the host before any launch; a bad argument
+ *     returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE
+ *     and launches nothing.  A failed launch returns MOE_ERR_CUDA.
+ *   - All work is asynchronous on `stream` (0 = legacy default stream).
+ *   - Device-side waits inside the kernels are bounded in time; when one
+ *     gives up, the kernel records MOE_ERR_TIMEOUT in the workspace status
+ *     word and returns; moe_check_device_status reports it.
+ *   - Results are deterministic: two calls on the same inputs give
+ *     bit-identical outputs (no atomics decide any order or sum).
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2,  /* valid shape this build does not run (e.g. E > 64) */
+    MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
+    MOE_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
+    MOE_ERR_TIMEOUT = 5       /* a bounded device wait gave up (see moe_check_device_status) */
+} moe_status_t;
+
+typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype_t;
+
+typedef enum {
+    MOE_ACT_SWIGLU = 0,     /* W_down( silu(x W_gate) * (x W_up) ) */
+    MOE_ACT_GELU_BIAS = 1   /* W2( gelu_erf(x W1 + b1) ) + b2 */
+} moe_act_t;
+
+/* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
+ * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
+typedef struct {
+    int64_t T;                 /* tokens (batch * sequence) */
+    int32_t d;                 /* model (hidden) dimension */
+    int32_t ffn;               /* expert intermediate dimension */
+    int32_t E;                 /* number of experts */
+    int32_t k;                 /* experts per token (top-k) */
+    int32_t dtype;             /* moe_dtype_t */
+    int32_t act;               /* moe_act_t */
+    double capacity_factor;    /* <= 0: no capacity limit (cap = T) */
+    float aux_alpha;           /* alpha of L_aux */
+    int32_t reserved;          /* must be 0 */
+} moe_config_t;
+
+/* Expert and router parameters (device, config dtype unless stated). */
+typedef struct {
+    const void* w_router;            /* [d, E] */
+    const float* router_logit_bias;  /* [E] float32 added to the logits before the softmax, or NULL */
+    const void* w_gate_or_w1;        /* [E, d, ffn]  SwiGLU W_gate | GELU W1 */
+    const void* w_up;                /* [E, d, ffn]  SwiGLU W_up   | NULL */
+    const void* w_down_or_w2;        /* [E, ffn, d]  SwiGLU W_down | GELU W2 */
+    const void* b1;                  /* [E, ffn] GELU only, else NULL */
+    const void* b2;                  /* [E, d]   GELU only, else NULL */
+} moe_weights_t;
+
+/* Outputs of moe_forward (device).  R_max = moe_max_rows(). */
+typedef struct {
+    void* out;             /* [T, d] layer output, token order */
+    int32_t* topk_idx;     /* [T, k] selected experts, best first (ties: lower id) */
+    float* topk_w;         /* [T, k] renormalised routing weights */
+    int32_t* counts;       /* [E] router selections per expert, before the capacity cut */
+    int32_t* offsets;      /* [E+1] start row of each expert's kept rows; offsets[E] = R */
+    int32_t* slot;         /* [T, k] row of assignment (t, j) in the expert-sorted buffers, or -1 if dropped */
+    int32_t* src_assign;   /* [R_max] t*k + j of each sorted row (first R entries written) */
+    float* f;              /* [E] f_e = counts_e / (T*k) */
+    float* p;              /* [E] p_e = mean over tokens of the full softmax */
+    float* l_aux;          /* [1] alpha * E * sum_e f_e p_e */
+    float* logits_out;     /* [T, E] router logits (bias included), or NULL */
+    float* probs_out;      /* [T, E] full softmax, or NULL */
+} moe_outputs_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status_t status);
+
+/* Per-expert capacity, evaluated on the host in double exactly as
+ * ceil(((double)T * k / E) * capacity_factor); capacity_factor <= 0 gives T.
+ * (MoE-basics §2.4, scaled by k because the buffer holds assignments.) */
+moe_status_t moe_capacity(const moe_config_t* cfg, int64_t* cap);
+
+/* Upper bound on dispatched rows: R_max = min(T*k, E*cap).  Size of the
+ * src_assign array and row count of x_perm / y_perm buffers. */
+moe_status_t moe_max_rows(const moe_config_t* cfg, int64_t* rows);
+
+/* Bytes of workspace the calls below need for this config (x_perm, h, y_perm,
+ * per-chunk partial histograms / probability sums, status word). */
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* Clear the workspace status word.  Call once after allocating a workspace
+ * (and after any MOE_ERR_TIMEOUT).  Asynchronous on `stream`. */
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Router + softmax + top-k + renormalisation (MoE-basics §2.1, §3.1;
+ * Llama-MoE §3.1).
+ *   x [T,d], w_router [d,E]; logit_bias [E] float32 or NULL.
+ *   logits_in [T,E] float32 or NULL: when given, these logits (bias already
+ *     included) replace x . W_r + bias -- used to feed both this library and a
+ *     reference identical logits.
+ *   topk_idx [T,k] int32, topk_w [T,k] float32 (outputs).
+ *   logits_out, probs_out [T,E] float32 or NULL (optional outputs).
+ * Top-k compares fp32 logits, lower id first on ties.  Needs a workspace. */
+moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router,
+                             const float* logit_bias, const float* logits_in,
+                             int32_t* topk_idx, float* topk_w, float* logits_out, float* probs_out,
+                             void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Capacity-bounded dispatch (MoE-basics §2.4; LLaMA4-MoE §2.4).
+ *   topk_idx [T,k] int32 in [0,E).  Outputs: counts [E], offsets [E+1],
+ *   slot [T,k], src_assign [R_max] (first offsets[E] entries), and
+ *   x_perm [R_max, d] whose row s is x[src_assign[s] / k].
+ * Assignment (t,j) has rank = number of earlier assignments (token-major
+ * order) to the same expert; it is kept iff rank < cap.  Needs a workspace. */
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                          int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* src_assign,
+                          void* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Expert FFNs over the expert-sorted rows (Loop-MoE §2.1 weight pool;
+ * MoE-basics §2.2, §3.1).  Rows [offsets[e], offsets[e+1]) of x_perm [R_max,d]
+ * go through expert e; y_perm [R_max, d] receives the results (rows >= R are
+ * not written).  bf16 runs on the tensor cores (fp32 accumulation; the
+ * intermediate activation is rounded to bf16 once); f32 runs in fp32 FMA.
+ * The intermediate [R_max, ffn] activation lives in the workspace. */
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_perm,
+                            const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* Weighted combine back to token order (LLaMA4-MoE §2.4; MoE-basics §3.1):
+ * out[t] = sum over j with slot[t,j] >= 0 of topk_w[t,j] * y_perm[slot[t,j]],
+ * accumulated in fp32 in ascending j; a token with every assignment dropped
+ * gets 0; surviving weights are not renormalised. */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* slot,
+                         const float* topk_w, void* out, cudaStream_t stream);
+
+/* Load-balance statistics (MoE-basics §2.3, §3.1; LLaMA4-MoE §3.2):
+ * f_e = counts_e / (T*k), p_e = (1/T) sum_t probs[t,e] (probs [T,E] float32,
+ * the full softmax), l_aux = alpha * E * sum_e f_e p_e.  T = 0 gives zeros. */
+moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const float* probs,
+                           float* f, float* p, float* l_aux, cudaStream_t stream);
+
+/* The whole layer forward: router, top-k, dispatch, expert FFNs, combine and
+ * aux statistics, six kernel launches on `stream`.  `logits_in` as in
+ * moe_router_topk (NULL in normal use). */
+moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
+                         const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* moe_forward, recording stage_events[i] on `stream` just before kernel
+ * launch i and stage_events[n] after the last launch, n =
+ * moe_forward_launch_count(cfg) (stage_events: caller-created CUDA events,
+ * at least n+1 of them).  For per-stage timing of the very same launch
+ * sequence; the computation is identical to moe_forward. */
+moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
+                                  const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream, cudaEvent_t* stage_events);
+
+/* moe_forward with the token activations in HOST memory: copies x_host
+ * (HOST, [T,d], pinned for asynchronous copies) to x_dev (device, [T,d]),
+ * runs moe_forward, and copies outputs->out to out_host (HOST, [T,d]) and
+ * outputs->l_aux to l_aux_host (HOST, 1 float).  Plain cudaMemcpyAsync on
+ * `stream`; the caller synchronises the stream before reading the host
+ * buffers. */
+moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_host,
+                                void* x_dev, moe_outputs_t* outputs, void* out_host, float* l_aux_host,
+                                void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the workspace status word.
+ * Returns MOE_ERR_TIMEOUT if a bounded device wait gave up since the last
+ * check (`*site`, if not NULL, receives the code of the first wait that gave
+ * up), MOE_ERR_CUDA if the synchronisation failed, else MOE_OK. */
+moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t* site);
+
+/* Time limit of every bounded device wait, in milliseconds (default 2000).
+ * Applies to launches made after the call; process-wide. */
+void moe_set_wait_timeout_ms(uint32_t ms);
+
+/* Self-test of the bounded-wait path: launches one block that waits on an
+ * mbarrier phase and on a workspace flag that nothing completes, each with a
+ * limit of `timeout_ms`.  Both waits give up; the status word then reports
+ * MOE_ERR_TIMEOUT through moe_check_device_status.  Used by the failure
+ * tests; faults and hangs nothing. */
+moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint32_t timeout_ms, cudaStream_t stream);
+
+/* Number of kernel launches moe_forward makes for this config. */
+int32_t moe_forward_launch_count(const moe_config_t* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,316 @@
+"""Python binding of libmoe, the B200 (sm_100a) MoE layer forward.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+of ``libmoe.so`` behind the C ABI declared in ``include/moe.h``.  PyTorch is
+used for device memory and streams.  There is no CPU fallback: if the
+library is missing or fails to load, the calls raise.
+
+The functions below carry the C names (``moe_forward``, ``moe_router_topk``,
+...) and take torch tensors (or None for optional pointers); ``MoELayer``
+bundles weights, outputs and workspace for the common case.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_DT_F32, MOE_DT_BF16 = 0, 1
+MOE_ACT_SWIGLU, MOE_ACT_GELU_BIAS = 0, 1
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)}")
+
+
+class MoEConfigC(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("ffn", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("reserved", ctypes.c_int32)]
+
+
+class MoEWeightsC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_router", "router_logit_bias", "w_gate_or_w1", "w_up", "w_down_or_w2", "b1", "b2")]
+
+
+class MoEOutputsC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("out", "topk_idx", "topk_w", "counts", "offsets", "slot", "src_assign", "f", "p", "l_aux",
+                 "logits_out", "probs_out")]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_CFG = ctypes.POINTER(MoEConfigC)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmoe.so not built ({LIB_PATH}); run `python -m mixture_experts_layer_37_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    st = ctypes.c_int
+    L.moe_status_string.argtypes = [st]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_capacity.argtypes = [_CFG, ctypes.POINTER(ctypes.c_int64)]
+    L.moe_max_rows.argtypes = [_CFG, ctypes.POINTER(ctypes.c_int64)]
+    L.moe_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
+    L.moe_router_topk.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.moe_dispatch.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.moe_expert_ffn.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
+    L.moe_aux_stats.argtypes = [_CFG, _P, _P, _P, _P, _P, _P]
+    L.moe_forward.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P,
+                              ctypes.c_size_t, _P]
+    L.moe_forward_profiled.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P,
+                                       ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_forward_hostio.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P, _P,
+                                     _P, ctypes.c_size_t, _P]
+    L.moe_check_device_status.argtypes = [_P, ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_uint32)]
+    L.moe_set_wait_timeout_ms.argtypes = [ctypes.c_uint32]
+    L.moe_set_wait_timeout_ms.restype = None
+    L.moe_selftest_bounded_wait.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint32, _P]
+    L.moe_forward_launch_count.argtypes = [_CFG]
+    for name in ("moe_capacity", "moe_max_rows", "moe_workspace_size", "moe_workspace_init", "moe_router_topk",
+                 "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
+                 "moe_forward_hostio", "moe_check_device_status", "moe_selftest_bounded_wait",
+                 "moe_forward_launch_count", "moe_forward_profiled"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size", "moe_workspace_init",
+                    "moe_router_topk", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_stats",
+                    "moe_forward", "moe_forward_hostio", "moe_check_device_status", "moe_set_wait_timeout_ms",
+                    "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled")
+
+
+# ---------------------------------------------------------------- config
+@dataclass(frozen=True)
+class MoEConfig:
+    T: int
+    d: int
+    ffn: int
+    E: int
+    k: int
+    dtype: str = "bf16"        # "bf16" | "f32"
+    act: str = "swiglu"        # "swiglu" | "gelu_bias"
+    capacity_factor: float = 1.25
+    aux_alpha: float = 0.01
+
+    def c(self) -> MoEConfigC:
+        return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
+                          MOE_DT_BF16 if self.dtype == "bf16" else MOE_DT_F32,
+                          MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
+                          float(self.capacity_factor), float(self.aux_alpha), 0)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @staticmethod
+    def of(wl) -> "MoEConfig":
+        """From a workload description (anything with the same field names)."""
+        return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def moe_capacity(cfg: MoEConfig) -> int:
+    v = ctypes.c_int64()
+    _check(lib().moe_capacity(ctypes.byref(cfg.c()), ctypes.byref(v)), "moe_capacity")
+    return v.value
+
+
+def moe_max_rows(cfg: MoEConfig) -> int:
+    v = ctypes.c_int64()
+    _check(lib().moe_max_rows(ctypes.byref(cfg.c()), ctypes.byref(v)), "moe_max_rows")
+    return v.value
+
+
+def moe_workspace_size(cfg: MoEConfig) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().moe_workspace_size(ctypes.byref(cfg.c()), ctypes.byref(v)), "moe_workspace_size")
+    return v.value
+
+
+class Workspace:
+    """A 1024-byte-aligned device buffer of moe_workspace_size() bytes, status word cleared."""
+
+    def __init__(self, cfg: MoEConfig, device="cuda", stream=None, nbytes: Optional[int] = None):
+        self.nbytes = moe_workspace_size(cfg) if nbytes is None else nbytes
+        self._buf = torch.empty(self.nbytes + 1024, dtype=torch.uint8, device=device)
+        off = (-self._buf.data_ptr()) % 1024
+        self.tensor = self._buf[off:off + self.nbytes]
+        self.ptr = self.tensor.data_ptr()
+        _check(lib().moe_workspace_init(self.ptr, self.nbytes, _stream(stream)), "moe_workspace_init")
+
+
+def moe_workspace_init(ws: Workspace, stream=None) -> None:
+    _check(lib().moe_workspace_init(ws.ptr, ws.nbytes, _stream(stream)), "moe_workspace_init")
+
+
+def moe_router_topk(cfg: MoEConfig, x, w_router, logit_bias, logits_in, topk_idx, topk_w, logits_out, probs_out,
+                    ws: Workspace, stream=None) -> None:
+    _check(lib().moe_router_topk(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(logit_bias), _ptr(logits_in),
+                                 _ptr(topk_idx), _ptr(topk_w), _ptr(logits_out), _ptr(probs_out), ws.ptr, ws.nbytes,
+                                 _stream(stream)), "moe_router_topk")
+
+
+def moe_dispatch(cfg: MoEConfig, x, topk_idx, counts, offsets, slot, src_assign, x_perm, ws: Workspace,
+                 stream=None) -> None:
+    _check(lib().moe_dispatch(ctypes.byref(cfg.c()), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(slot),
+                              _ptr(src_assign), _ptr(x_perm), ws.ptr, ws.nbytes, _stream(stream)), "moe_dispatch")
+
+
+def _weights_c(w: dict) -> MoEWeightsC:
+    g = lambda n: _ptr(w.get(n))  # noqa: E731
+    return MoEWeightsC(g("w_router"), g("router_bias"), g("w_gate") if "w_gate" in w else g("w1"), g("w_up"),
+                       g("w_down") if "w_down" in w else g("w2"), g("b1"), g("b2"))
+
+
+def moe_expert_ffn(cfg: MoEConfig, weights: dict, x_perm, offsets, y_perm, ws: Workspace, stream=None) -> None:
+    wc = _weights_c(weights)
+    _check(lib().moe_expert_ffn(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x_perm), _ptr(offsets), _ptr(y_perm),
+                                ws.ptr, ws.nbytes, _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(cfg: MoEConfig, y_perm, slot, topk_w, out, stream=None) -> None:
+    _check(lib().moe_combine(ctypes.byref(cfg.c()), _ptr(y_perm), _ptr(slot), _ptr(topk_w), _ptr(out),
+                             _stream(stream)), "moe_combine")
+
+
+def moe_aux_stats(cfg: MoEConfig, counts, probs, f, p, l_aux, stream=None) -> None:
+    _check(lib().moe_aux_stats(ctypes.byref(cfg.c()), _ptr(counts), _ptr(probs), _ptr(f), _ptr(p), _ptr(l_aux),
+                               _stream(stream)), "moe_aux_stats")
+
+
+_OUT_FIELDS = ("out", "topk_idx", "topk_w", "counts", "offsets", "slot", "src_assign", "f", "p", "l_aux",
+               "logits_out", "probs_out")
+
+
+def _outputs_c(o: dict) -> MoEOutputsC:
+    return MoEOutputsC(*[_ptr(o.get(n)) for n in _OUT_FIELDS])
+
+
+def allocate_outputs(cfg: MoEConfig, device="cuda", with_logits: bool = False, with_probs: bool = False) -> dict:
+    T, E, k = cfg.T, cfg.E, cfg.k
+    o = {
+        "out": torch.empty((T, cfg.d), dtype=cfg.torch_dtype, device=device),
+        "topk_idx": torch.empty((T, k), dtype=torch.int32, device=device),
+        "topk_w": torch.empty((T, k), dtype=torch.float32, device=device),
+        "counts": torch.empty(E, dtype=torch.int32, device=device),
+        "offsets": torch.empty(E + 1, dtype=torch.int32, device=device),
+        "slot": torch.empty((T, k), dtype=torch.int32, device=device),
+        "src_assign": torch.empty(max(moe_max_rows(cfg), 1), dtype=torch.int32, device=device),
+        "f": torch.empty(E, dtype=torch.float32, device=device),
+        "p": torch.empty(E, dtype=torch.float32, device=device),
+        "l_aux": torch.empty(1, dtype=torch.float32, device=device),
+    }
+    if with_logits:
+        o["logits_out"] = torch.empty((T, E), dtype=torch.float32, device=device)
+    if with_probs:
+        o["probs_out"] = torch.empty((T, E), dtype=torch.float32, device=device)
+    return o
+
+
+def moe_forward(cfg: MoEConfig, weights: dict, x, outputs: dict, ws: Workspace, logits_in=None, stream=None) -> None:
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    _check(lib().moe_forward(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x), _ptr(logits_in), ctypes.byref(oc),
+                             ws.ptr, ws.nbytes, _stream(stream)), "moe_forward")
+
+
+def moe_forward_profiled(cfg: MoEConfig, weights: dict, x, outputs: dict, ws: Workspace, events: list,
+                         logits_in=None, stream=None) -> None:
+    """moe_forward recording torch.cuda.Event objects `events` (n+1 of them,
+    n = moe_forward_launch_count) around each kernel launch on `stream`."""
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    _check(lib().moe_forward_profiled(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x), _ptr(logits_in),
+                                      ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream), arr),
+           "moe_forward_profiled")
+
+
+def moe_forward_hostio(cfg: MoEConfig, weights: dict, x_host, x_dev, outputs: dict, out_host, l_aux_host,
+                       ws: Workspace, stream=None) -> None:
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    _check(lib().moe_forward_hostio(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x_host), _ptr(x_dev),
+                                    ctypes.byref(oc), _ptr(out_host), _ptr(l_aux_host), ws.ptr, ws.nbytes,
+                                    _stream(stream)), "moe_forward_hostio")
+
+
+def moe_check_device_status(ws: Workspace, stream=None) -> tuple:
+    """(status, site): synchronises the stream, reads and clears the status word."""
+    site = ctypes.c_uint32(0)
+    st = lib().moe_check_device_status(ws.ptr, ws.nbytes, _stream(stream), ctypes.byref(site))
+    return st, site.value
+
+
+def moe_set_wait_timeout_ms(ms: int) -> None:
+    lib().moe_set_wait_timeout_ms(int(ms))
+
+
+def moe_selftest_bounded_wait(ws: Workspace, timeout_ms: int, stream=None) -> None:
+    _check(lib().moe_selftest_bounded_wait(ws.ptr, ws.nbytes, int(timeout_ms), _stream(stream)),
+           "moe_selftest_bounded_wait")
+
+
+def moe_forward_launch_count(cfg: MoEConfig) -> int:
+    return lib().moe_forward_launch_count(ctypes.byref(cfg.c()))
+
+
+# ---------------------------------------------------------------- layer
+class MoELayer:
+    """Weights + preallocated outputs and workspace for repeated forwards."""
+
+    def __init__(self, cfg: MoEConfig, weights: dict, device="cuda", with_logits=False, with_probs=False):
+        self.cfg = cfg
+        self.weights = weights
+        self.outputs = allocate_outputs(cfg, device, with_logits, with_probs)
+        self.ws = Workspace(cfg, device)
+
+    def forward(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None, stream=None) -> dict:
+        moe_forward(self.cfg, self.weights, x, self.outputs, self.ws, logits_in, stream)
+        return self.outputs
+
+    def check(self, stream=None) -> None:
+        st, site = moe_check_device_status(self.ws, stream)
+        if st != MOE_OK:
+            raise MoEError(st, f"device status (site 0x{site:x})")

@@ -1,0 +1,98 @@
+// Host-side launch interfaces between the C ABI (moe_api.cu) and the kernel
+// translation units.  Internal to libmoe.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct RouterArgs {
+    const void* x;           // [T, d] act dtype
+    const void* w_router;    // [d, E] act dtype
+    const float* bias;       // [E] or null
+    const float* logits_in;  // [T, E] or null
+    int32_t* topk_idx;       // [T, k]
+    float* topk_w;           // [T, k]
+    float* logits_out;       // [T, E] or null
+    float* probs_out;        // [T, E] or null
+    int32_t* hist;           // [nchunk, E] per-chunk expert histogram
+    double* psum;            // [nchunk, E] per-chunk sum of probabilities
+    int64_t T;
+    int d, E, k;
+};
+cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
+
+struct ScanArgs {
+    const int32_t* hist;   // [nchunk, E]
+    const double* psum;    // [nchunk, E] or null (no aux stats)
+    int32_t* chunk_base;   // [nchunk, E] out
+    int32_t* counts;       // [E] out
+    int32_t* offsets;      // [E+1] out
+    float* f;              // [E] out or null
+    float* p;              // [E] out or null
+    float* l_aux;          // [1] out or null
+    int64_t T;
+    int nchunk, E, k, cap;
+    float alpha;
+};
+cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s);
+cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s);
+
+struct ScatterArgs {
+    const int32_t* topk_idx;    // [T, k]
+    const int32_t* chunk_base;  // [nchunk, E]
+    const int32_t* offsets;     // [E+1]
+    int32_t* slot;              // [T, k]
+    int32_t* src_assign;        // [R_max]
+    const void* x;              // [T, d]
+    void* x_perm;               // [R_max, d]
+    int64_t T;
+    int E, k, cap;
+    int row_bytes;              // d * element size (multiple of 16)
+};
+cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+    const void* y_perm;    // [R_max, d]
+    const int32_t* slot;   // [T, k]
+    const float* topk_w;   // [T, k]
+    void* out;             // [T, d]
+    int64_t T;
+    int d, k;
+};
+cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s);
+cudaError_t launch_aux_from_probs(const int32_t* counts, const float* probs, float* f, float* p, float* l_aux,
+                                  int64_t T, int E, int k, float alpha, cudaStream_t s);
+
+// Expert FFN (grouped GEMMs over the expert-sorted rows).
+struct FfnArgs {
+    int act;                 // 0 swiglu, 1 gelu+bias
+    int E, d, ffn;
+    int64_t rows_cap;        // R_max (rows allocated in x_perm / h / y_perm)
+    const int32_t* offsets;  // [E+1]
+    const void* x_perm;      // [rows_cap, d]
+    void* h;                 // [rows_cap, ffn] (workspace)
+    void* y_perm;            // [rows_cap, d]
+    const void* w1;          // [E, d, ffn] (gate or W1)
+    const void* w_up;        // [E, d, ffn] or null
+    const void* w2;          // [E, ffn, d]
+    const void* b1;          // [E, ffn] or null
+    const void* b2;          // [E, d] or null
+    DevStatus st;
+    cudaEvent_t between;     // recorded between the two GEMM launches, or null
+};
+// bf16: tcgen05 grouped GEMMs (two launches).  Returns cudaErrorInvalidValue
+// when a tensor map cannot be encoded.
+cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s);
+// f32: SIMT FMA grouped GEMMs (two launches).
+cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
+
+cudaError_t launch_selftest_wait(DevStatus st, cudaStream_t s);
+
+int sm_count();
+
+}  // namespace moe

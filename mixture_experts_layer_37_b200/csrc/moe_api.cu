@@ -1,0 +1,449 @@
+// libmoe C ABI: argument validation, capacity and workspace planning, and the
+// kernel launch sequence of the MoE layer forward.  No allocation, no host
+// synchronisation (except moe_check_device_status), no CPU fallback.
+#include <math.h>
+#include <string.h>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        return n > 0 ? n : 1;
+    }
+    if (cached[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 1;
+    }
+    return cached[dev];
+}
+
+}  // namespace moe
+
+namespace {
+
+using namespace moe;
+
+uint32_t g_timeout_ms = 2000;
+
+constexpr size_t kStatusBytes = 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+size_t elem_size(const moe_config_t* c) { return c->dtype == MOE_DT_BF16 ? 2 : 4; }
+
+moe_status_t check_config(const moe_config_t* c) {
+    if (c == nullptr) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->d <= 0 || c->ffn <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+    if (c->dtype != MOE_DT_F32 && c->dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
+    if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->reserved != 0) return MOE_ERR_INVALID_ARG;
+    if (c->E > kMaxExperts || c->k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+    if (c->T * (int64_t)c->k >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    if (c->dtype == MOE_DT_BF16) {
+        if (c->d % 64 != 0 || c->ffn % 64 != 0) return MOE_ERR_UNSUPPORTED;
+        if ((int64_t)c->E * c->d >= ((int64_t)1 << 31) || (int64_t)c->E * c->ffn >= ((int64_t)1 << 31))
+            return MOE_ERR_UNSUPPORTED;
+    } else {
+        if (c->d % 4 != 0 || c->ffn % 4 != 0) return MOE_ERR_UNSUPPORTED;
+    }
+    return MOE_OK;
+}
+
+// Formula value of the capacity (may exceed T) and the clamped value the
+// kernels use (an expert can receive at most T assignments).
+int64_t capacity_formula(const moe_config_t* c) {
+    if (!(c->capacity_factor > 0.0)) return c->T;
+    const double v = ceil(((double)c->T * (double)c->k / (double)c->E) * c->capacity_factor);
+    if (v >= 9.0e18) return INT64_MAX;
+    return (int64_t)v;
+}
+int64_t capacity_used(const moe_config_t* c) {
+    const int64_t cap = capacity_formula(c);
+    return cap < c->T ? cap : c->T;
+}
+int64_t max_rows(const moe_config_t* c) {
+    const int64_t cap = capacity_used(c);
+    const int64_t a = c->T * c->k, b = (int64_t)c->E * cap;
+    return a < b ? a : b;
+}
+
+struct Plan {
+    int nchunk;
+    int64_t rows;
+    size_t hist, psum, base, xperm, h, yperm, total;
+};
+
+Plan plan_of(const moe_config_t* c) {
+    Plan p;
+    p.nchunk = (int)((c->T + kChunkTokens - 1) / kChunkTokens);
+    p.rows = max_rows(c);
+    const size_t s = elem_size(c);
+    const size_t E = (size_t)c->E;
+    size_t off = kStatusBytes;
+    p.hist = off;
+    off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
+    p.psum = off;
+    off = align_up(off + (size_t)p.nchunk * E * 8, 1024);
+    p.base = off;
+    off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
+    p.xperm = off;
+    off = align_up(off + (size_t)p.rows * c->d * s, 1024);
+    p.h = off;
+    off = align_up(off + (size_t)p.rows * c->ffn * s, 1024);
+    p.yperm = off;
+    off = align_up(off + (size_t)p.rows * c->d * s, 1024);
+    p.total = off;
+    return p;
+}
+
+moe_status_t check_ws(const moe_config_t* c, const void* ws, size_t ws_bytes, Plan* p) {
+    *p = plan_of(c);
+    if (ws == nullptr || ws_bytes < p->total) return MOE_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 1023u) != 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+DevStatus status_of(void* ws) {
+    DevStatus st;
+    st.word = static_cast<uint32_t*>(ws);
+    st.timeout_ns = (uint64_t)g_timeout_ms * 1000000ull;
+    return st;
+}
+
+uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status_t check_weights(const moe_config_t* c, const moe_weights_t* w, bool need_router, bool need_experts) {
+    if (w == nullptr) return MOE_ERR_INVALID_ARG;
+    if (need_router && (w->w_router == nullptr || !aligned16(w->w_router))) return MOE_ERR_INVALID_ARG;
+    if (need_experts) {
+        if (w->w_gate_or_w1 == nullptr || w->w_down_or_w2 == nullptr) return MOE_ERR_INVALID_ARG;
+        if (!aligned16(w->w_gate_or_w1) || !aligned16(w->w_down_or_w2)) return MOE_ERR_INVALID_ARG;
+        if (c->act == MOE_ACT_SWIGLU) {
+            if (w->w_up == nullptr || !aligned16(w->w_up)) return MOE_ERR_INVALID_ARG;
+        } else {
+            if (w->b1 == nullptr || w->b2 == nullptr) return MOE_ERR_INVALID_ARG;
+        }
+    }
+    return MOE_OK;
+}
+
+moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_router, const float* bias,
+                        const float* logits_in, int32_t* idx, float* w, float* logits_out, float* probs_out,
+                        void* ws, const Plan& pl, cudaStream_t s) {
+    RouterArgs a;
+    a.x = x;
+    a.w_router = w_router;
+    a.bias = bias;
+    a.logits_in = logits_in;
+    a.topk_idx = idx;
+    a.topk_w = w;
+    a.logits_out = logits_out;
+    a.probs_out = probs_out;
+    a.hist = reinterpret_cast<int32_t*>(at(ws, pl.hist));
+    a.psum = reinterpret_cast<double*>(at(ws, pl.psum));
+    a.T = c->T;
+    a.d = c->d;
+    a.E = c->E;
+    a.k = c->k;
+    return from_cuda(launch_router(a, c->dtype == MOE_DT_BF16, s));
+}
+
+moe_status_t run_scan_scatter(const moe_config_t* c, const void* x, const int32_t* idx, int32_t* counts,
+                              int32_t* offsets, int32_t* slot, int32_t* src_assign, void* x_perm, float* f, float* p,
+                              float* l_aux, bool with_stats, void* ws, const Plan& pl, cudaStream_t s,
+                              cudaEvent_t between = nullptr) {
+    ScanArgs sa;
+    sa.hist = reinterpret_cast<const int32_t*>(at(ws, pl.hist));
+    sa.psum = with_stats ? reinterpret_cast<const double*>(at(ws, pl.psum)) : nullptr;
+    sa.chunk_base = reinterpret_cast<int32_t*>(at(ws, pl.base));
+    sa.counts = counts;
+    sa.offsets = offsets;
+    sa.f = f;
+    sa.p = p;
+    sa.l_aux = l_aux;
+    sa.T = c->T;
+    sa.nchunk = pl.nchunk;
+    sa.E = c->E;
+    sa.k = c->k;
+    sa.cap = (int)capacity_used(c);
+    sa.alpha = c->aux_alpha;
+    cudaError_t e = launch_dispatch_scan(sa, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (sa.nchunk == 0) return MOE_OK;
+    if (between != nullptr && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
+    ScatterArgs xa;
+    xa.topk_idx = idx;
+    xa.chunk_base = sa.chunk_base;
+    xa.offsets = offsets;
+    xa.slot = slot;
+    xa.src_assign = src_assign;
+    xa.x = x;
+    xa.x_perm = x_perm;
+    xa.T = c->T;
+    xa.E = c->E;
+    xa.k = c->k;
+    xa.cap = sa.cap;
+    xa.row_bytes = (int)(c->d * elem_size(c));
+    return from_cuda(launch_dispatch_scatter(xa, s));
+}
+
+moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* x_perm, const int32_t* offsets,
+                     void* y_perm, void* ws, const Plan& pl, cudaStream_t s, cudaEvent_t between = nullptr) {
+    FfnArgs f;
+    f.act = c->act;
+    f.E = c->E;
+    f.d = c->d;
+    f.ffn = c->ffn;
+    f.rows_cap = pl.rows;
+    f.offsets = offsets;
+    f.x_perm = x_perm;
+    f.h = at(ws, pl.h);
+    f.y_perm = y_perm;
+    f.w1 = w->w_gate_or_w1;
+    f.w_up = w->w_up;
+    f.w2 = w->w_down_or_w2;
+    f.b1 = w->b1;
+    f.b2 = w->b2;
+    f.st = status_of(ws);
+    f.between = between;
+    return from_cuda(c->dtype == MOE_DT_BF16 ? launch_ffn_bf16_sm100(f, s) : launch_ffn_f32(f, s));
+}
+
+moe_status_t run_combine(const moe_config_t* c, const void* y_perm, const int32_t* slot, const float* w, void* out,
+                         cudaStream_t s) {
+    CombineArgs a;
+    a.y_perm = y_perm;
+    a.slot = slot;
+    a.topk_w = w;
+    a.out = out;
+    a.T = c->T;
+    a.d = c->d;
+    a.k = c->k;
+    return from_cuda(launch_combine(a, c->dtype == MOE_DT_BF16, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside what this build runs";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or smaller than moe_workspace_size";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_capacity(const moe_config_t* cfg, int64_t* cap) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (cap == nullptr) return MOE_ERR_INVALID_ARG;
+    *cap = capacity_formula(cfg);
+    return MOE_OK;
+}
+
+moe_status_t moe_max_rows(const moe_config_t* cfg, int64_t* rows) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (rows == nullptr) return MOE_ERR_INVALID_ARG;
+    *rows = max_rows(cfg);
+    return MOE_OK;
+}
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+    *bytes = plan_of(cfg).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (ws == nullptr || ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    return from_cuda(cudaMemsetAsync(ws, 0, kStatusBytes, stream));
+}
+
+moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
+                             const float* logits_in, int32_t* topk_idx, float* topk_w, float* logits_out,
+                             float* probs_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+    if (logits_in == nullptr) {
+        if (x == nullptr || w_router == nullptr || !aligned16(x) || !aligned16(w_router)) return MOE_ERR_INVALID_ARG;
+    }
+    Plan pl;
+    if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;
+    return run_router(cfg, x, w_router, logit_bias, logits_in, topk_idx, topk_w, logits_out, probs_out, ws, pl, stream);
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
+                          int32_t* offsets, int32_t* slot, int32_t* src_assign, void* x_perm, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || topk_idx == nullptr || slot == nullptr || src_assign == nullptr ||
+                       x_perm == nullptr || !aligned16(x) || !aligned16(x_perm)))
+        return MOE_ERR_INVALID_ARG;
+    Plan pl;
+    if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
+    if (launch_dispatch_hist(topk_idx, reinterpret_cast<int32_t*>(at(ws, pl.hist)), cfg->T, cfg->E, cfg->k, stream) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
+    return run_scan_scatter(cfg, x, topk_idx, counts, offsets, slot, src_assign, x_perm, nullptr, nullptr, nullptr,
+                            false, ws, pl, stream);
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_perm,
+                            const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_weights(cfg, weights, false, true)) != MOE_OK) return st;
+    if (offsets == nullptr || x_perm == nullptr || y_perm == nullptr || !aligned16(x_perm) || !aligned16(y_perm))
+        return MOE_ERR_INVALID_ARG;
+    Plan pl;
+    if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
+    if (pl.rows == 0) return MOE_OK;
+    return run_ffn(cfg, weights, x_perm, offsets, y_perm, ws, pl, stream);
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* slot, const float* topk_w,
+                         void* out, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;
+    if (y_perm == nullptr || slot == nullptr || topk_w == nullptr || out == nullptr || !aligned16(y_perm) ||
+        !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    return run_combine(cfg, y_perm, slot, topk_w, out, stream);
+}
+
+moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const float* probs, float* f, float* p,
+                           float* l_aux, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (counts == nullptr || f == nullptr || p == nullptr || l_aux == nullptr) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && probs == nullptr) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_aux_from_probs(counts, probs, f, p, l_aux, cfg->T, cfg->E, cfg->k, cfg->aux_alpha, stream));
+}
+
+static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
+                                 const float* logits_in, moe_outputs_t* o, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream, cudaEvent_t* ev) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_weights(cfg, weights, logits_in == nullptr, true)) != MOE_OK) return st;
+    if (o == nullptr || o->counts == nullptr || o->offsets == nullptr || o->f == nullptr || o->p == nullptr ||
+        o->l_aux == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->out == nullptr || !aligned16(o->out) ||
+                       o->topk_idx == nullptr || o->topk_w == nullptr || o->slot == nullptr ||
+                       o->src_assign == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    Plan pl;
+    if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
+    int n = 0;
+    auto mark = [&]() -> bool { return ev == nullptr || cudaEventRecord(ev[n++], stream) == cudaSuccess; };
+    if (cfg->T > 0) {
+        if (!mark()) return MOE_ERR_CUDA;
+        st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
+                        o->logits_out, o->probs_out, ws, pl, stream);
+        if (st != MOE_OK) return st;
+    }
+    void* x_perm = at(ws, pl.xperm);
+    void* y_perm = at(ws, pl.yperm);
+    if (!mark()) return MOE_ERR_CUDA;
+    st = run_scan_scatter(cfg, x, o->topk_idx, o->counts, o->offsets, o->slot, o->src_assign, x_perm, o->f, o->p,
+                          o->l_aux, true, ws, pl, stream, (ev && cfg->T > 0) ? ev[n++] : nullptr);
+    if (st != MOE_OK) return st;
+    if (cfg->T == 0) return mark() ? MOE_OK : MOE_ERR_CUDA;
+    if (!mark()) return MOE_ERR_CUDA;
+    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr);
+    if (st != MOE_OK) return st;
+    if (!mark()) return MOE_ERR_CUDA;
+    st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
+    if (st != MOE_OK) return st;
+    return mark() ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, const float* logits_in,
+                         moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return forward_impl(cfg, weights, x, logits_in, o, ws, ws_bytes, stream, nullptr);
+}
+
+moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
+                                  const float* logits_in, moe_outputs_t* o, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream, cudaEvent_t* stage_events) {
+    if (stage_events == nullptr) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg, weights, x, logits_in, o, ws, ws_bytes, stream, stage_events);
+}
+
+moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_host,
+                                void* x_dev, moe_outputs_t* o, void* out_host, float* l_aux_host, void* ws,
+                                size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (o == nullptr || l_aux_host == nullptr) return MOE_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)cfg->T * cfg->d * elem_size(cfg);
+    if (cfg->T > 0 && (x_host == nullptr || x_dev == nullptr || out_host == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (bytes && cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    st = moe_forward(cfg, weights, x_dev, nullptr, o, ws, ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    if (bytes && cudaMemcpyAsync(out_host, o->out, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(l_aux_host, o->l_aux, sizeof(float), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t* site) {
+    if (ws == nullptr || ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t words[3] = {0, 0, 0};
+    if (cudaMemcpyAsync(words, ws, sizeof(words), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (site) *site = words[1];
+    if (words[0] & kErrTimeout) {
+        if (cudaMemsetAsync(ws, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_ERR_TIMEOUT;
+    }
+    return MOE_OK;
+}
+
+void moe_set_wait_timeout_ms(uint32_t ms) { g_timeout_ms = ms == 0 ? 1 : ms; }
+
+moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint32_t timeout_ms, cudaStream_t stream) {
+    if (ws == nullptr || ws_bytes < kStatusBytes) return MOE_ERR_WORKSPACE;
+    DevStatus st;
+    st.word = static_cast<uint32_t*>(ws);
+    st.timeout_ns = (uint64_t)(timeout_ms == 0 ? 1 : timeout_ms) * 1000000ull;
+    return from_cuda(launch_selftest_wait(st, stream));
+}
+
+int32_t moe_forward_launch_count(const moe_config_t* cfg) {
+    if (check_config(cfg) != MOE_OK) return 0;
+    if (cfg->T == 0) return 1;
+    return 6;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, validates arguments on the host before any launch, and
+computes the capacity exactly as the oracle does."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import mixture_experts_layer_37_b200 as M
+from oracle import moe_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixture_experts_layer_37_b200 import build
+    build.build()
+    return M.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 15, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(names) == set(M.EXPORTED_SYMBOLS)
+
+
+def test_config_struct_layout_matches_header():
+    assert ctypes.sizeof(M.MoEConfigC) == 48
+    assert M.MoEConfigC.capacity_factor.offset == 32
+    assert ctypes.sizeof(M.MoEWeightsC) == 7 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
+
+
+@pytest.mark.parametrize("T,k,E,cf", [(64, 2, 4, 1.25), (4096, 2, 8, 1.25), (8192, 2, 8, 1.25), (32768, 2, 32, 1.0),
+                                      (64, 2, 64, 0.0), (10, 2, 3, 1.1), (4, 1, 1, 0.5), (1000, 3, 7, 0.9),
+                                      (333, 2, 5, 1.0 / 3.0), (1, 1, 1, 1e-9), (12345, 8, 64, 2.5), (7, 2, 3, -1.0)])
+def test_capacity_matches_oracle(lib, T, k, E, cf):
+    cfg = M.MoEConfig(T=T, d=64, ffn=64, E=E, k=k, capacity_factor=cf)
+    assert M.moe_capacity(cfg) == O.capacity(T, k, E, cf)
+    cap = min(O.capacity(T, k, E, cf), T)
+    assert M.moe_max_rows(cfg) == min(T * k, E * cap)
+
+
+def test_capacity_random_sweep(lib):
+    rng = np.random.default_rng(9)
+    for _ in range(2000):
+        E = int(rng.integers(1, 65))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        T = int(rng.integers(0, 200000))
+        cf = float(rng.choice([rng.uniform(0.01, 4.0), round(rng.uniform(0.5, 2), 2), 1.0, 1.25, 0.0]))
+        cfg = M.MoEConfig(T=T, d=64, ffn=64, E=E, k=k, capacity_factor=cf)
+        assert M.moe_capacity(cfg) == O.capacity(T, k, E, cf)
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_invalid_configs_rejected_on_host(lib):
+    size = ctypes.c_size_t()
+    bad = [
+        (dict(E=65, k=2), M.MOE_ERR_UNSUPPORTED),
+        (dict(E=4, k=5), M.MOE_ERR_INVALID_ARG),
+        (dict(E=16, k=9), M.MOE_ERR_UNSUPPORTED),
+        (dict(d=100), M.MOE_ERR_UNSUPPORTED),          # bf16 needs d % 64
+        (dict(ffn=96), M.MOE_ERR_UNSUPPORTED),
+        (dict(T=-1), M.MOE_ERR_INVALID_ARG),
+        (dict(E=0), M.MOE_ERR_INVALID_ARG),
+        (dict(capacity_factor=float("nan")), M.MOE_ERR_INVALID_ARG),
+        (dict(T=2 ** 30, k=2), M.MOE_ERR_UNSUPPORTED),  # T*k must stay below 2^31
+    ]
+    for kw, want in bad:
+        base = dict(T=128, d=128, ffn=128, E=8, k=2)
+        base.update(kw)
+        cfg = M.MoEConfig(**base).c()
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == want, kw
+    f32 = M.MoEConfig(T=8, d=100, ffn=12, E=2, k=1, dtype="f32").c()
+    assert lib.moe_workspace_size(ctypes.byref(f32), ctypes.byref(size)) == M.MOE_OK
+    cfg = M.MoEConfig(T=8, d=128, ffn=128, E=4, k=2).c()
+    cfg.dtype = 7
+    assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
+
+
+def test_null_and_workspace_errors_launch_nothing(lib):
+    """Bad pointers and short workspaces are refused before any CUDA call, so
+    these calls are safe without a GPU."""
+    cfg = M.MoEConfig(T=128, d=128, ffn=128, E=8, k=2)
+    c = cfg.c()
+    w = M.MoEWeightsC()
+    o = M.MoEOutputsC()
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), None, None, ctypes.byref(o), None, 0, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(ctypes.byref(c), None, None, None, None, None, 0, None) == M.MOE_ERR_INVALID_ARG
+    # well-formed pointers (never dereferenced) but no workspace
+    fake = ctypes.c_void_p(1 << 40)
+    w = M.MoEWeightsC(fake, None, fake, fake, fake, None, None)
+    o = M.MoEOutputsC(*([fake] * 10 + [None, None]))
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, ctypes.byref(o), None, 0, None) == \
+        M.MOE_ERR_WORKSPACE
+    need = M.moe_workspace_size(cfg)
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, ctypes.byref(o), fake, need - 1, None) == \
+        M.MOE_ERR_WORKSPACE
+    # misaligned activation pointer
+    mis = ctypes.c_void_p((1 << 40) + 8)
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), mis, None, ctypes.byref(o), fake, need, None) == \
+        M.MOE_ERR_INVALID_ARG
+    # swiglu without w_up
+    w2 = M.MoEWeightsC(fake, None, fake, None, fake, None, None)
+    assert lib.moe_expert_ffn(ctypes.byref(c), ctypes.byref(w2), fake, fake, fake, fake, need, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_topk(ctypes.byref(c), fake, fake, None, None, None, fake, None, None, fake, need,
+                               None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(ctypes.byref(c), None, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_aux_stats(ctypes.byref(c), None, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_size_accounts_for_buffers(lib):
+    cfg = M.MoEConfig(T=4096, d=2048, ffn=4096, E=8, k=2)
+    rows = M.moe_max_rows(cfg)
+    assert rows == 8192
+    ws = M.moe_workspace_size(cfg)
+    assert ws >= rows * (2048 * 2 * 2 + 4096 * 2)
+    assert M.moe_forward_launch_count(cfg) == 6
+    assert M.moe_forward_launch_count(M.MoEConfig(T=0, d=64, ffn=64, E=2, k=1)) == 1
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert M.moe_status_string(s).startswith("MOE_")
+    assert "UNKNOWN" in M.moe_status_string(99)
