@@ -154,6 +154,22 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
                           int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* src_assign,
                           void* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Allocation-free variant of moe_dispatch, for callers that cannot allocate
+ * device memory (for instance a plugin that is handed only its input and
+ * output buffers by a host framework owning all allocations, or a loop that
+ * must not allocate after start-up) and so cannot supply a workspace.  The
+ * pages have no counterpart: this is a property of the library, not of the
+ * method.  Same arguments, results and errors as moe_dispatch, minus the
+ * workspace.  Its scratch (per-chunk histograms and rank bases) is a fixed
+ * 512 KiB array in the library's device memory on every GPU that loads it;
+ * shapes with ceil(T/64)*E > 65536 return MOE_ERR_UNSUPPORTED.  The first
+ * call on a device looks up that array's address and should come before any
+ * stream capture.  All calls on a device share the array: calls that overlap
+ * on the GPU race and must be serialised by the caller. */
+moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                  int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* src_assign,
+                                  void* x_perm, cudaStream_t stream);
+
 /* Expert FFNs over the expert-sorted rows (Loop-MoE §2.1 weight pool;
  * MoE-basics §2.2, §3.1).  Rows [offsets[e], offsets[e+1]) of x_perm [R_max,d]
  * go through expert e; y_perm [R_max, d] receives the results (rows >= R are

@@ -97,7 +97,8 @@ def lib() -> ctypes.CDLL:
 EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size", "moe_workspace_init",
                     "moe_router_topk", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_stats",
                     "moe_forward", "moe_forward_hostio", "moe_check_device_status", "moe_set_wait_timeout_ms",
-                    "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled")
+                    "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled",
+                    "moe_dispatch_noalloc")
 
 
 # ---------------------------------------------------------------- config
@@ -314,3 +315,15 @@ class MoELayer:
         st, site = moe_check_device_status(self.ws, stream)
         if st != MOE_OK:
             raise MoEError(st, f"device status (site 0x{site:x})")
+
+
+def moe_dispatch_noalloc(cfg: MoEConfig, x, topk_idx, counts, offsets, slot, src_assign, x_perm, stream=None) -> None:
+    """moe_dispatch without a workspace, for callers that cannot allocate device
+    memory: the scratch lives in a fixed array inside the library (see
+    include/moe.h for the size limit and the rule that calls must not overlap)."""
+    L = lib()
+    f = L.moe_dispatch_noalloc
+    f.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]
+    f.restype = ctypes.c_int
+    _check(f(ctypes.byref(cfg.c()), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(slot),
+             _ptr(src_assign), _ptr(x_perm), _stream(stream)), "moe_dispatch_noalloc")
