@@ -4,7 +4,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
 
 One step = one whole layer forward (router, top-k, dispatch, expert FFNs,
-combine, aux statistics: six kernel launches) over one batch of the workload,
+combine, aux statistics: five kernel launches) over one batch of the workload,
 inputs resident in HBM.  A 256 MiB buffer (twice the L2) is written between
 steps, outside the timed events, so every step starts with a cold L2.  Each
 step is timed with CUDA events on the launching stream; the per-stage events
@@ -236,7 +236,8 @@ def run_native(a):
 
     # ---------------- roofline of the dominant kernel
     R = int(layer.outputs["offsets"][-1].item())
-    names = ["router", "scan", "scatter", "gemm1", "gemm2", "combine"]
+    names = ["router", "scatter", "gemm1", "gemm2", "combine"]  # router includes the fused dispatch scan
+    assert len(names) == nl, (names, nl)
     mean_stage = stage_ms.mean(axis=0)
     pk, pk_src = peaks()
     bpe = 2 if wl.dtype == "bf16" else 4
@@ -244,7 +245,6 @@ def run_native(a):
     gemm2_flops = 2 * wl.d * wl.ffn * R
     algo = {
         "router": ("hbm", wl.T * wl.d * bpe + wl.d * wl.E * bpe + wl.T * wl.k * 8),
-        "scan": ("hbm", 0),
         "scatter": ("hbm", 2 * R * wl.d * bpe + wl.T * wl.k * 4 * 3),
         "gemm1": ("tensor", gemm1_flops),
         "gemm2": ("tensor", gemm2_flops),

@@ -161,8 +161,9 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  * pages have no counterpart: this is a property of the library, not of the
  * method.  Same arguments, results and errors as moe_dispatch, minus the
  * workspace.  Its scratch (per-chunk histograms and rank bases) is a fixed
- * 512 KiB array in the library's device memory on every GPU that loads it;
- * shapes with ceil(T/64)*E > 65536 return MOE_ERR_UNSUPPORTED.  The first
+ * 1 MiB array in the library's device memory on every GPU that loads it;
+ * shapes with ceil(T/32)*E > 131072 (E = 64: T > 65536) return
+ * MOE_ERR_UNSUPPORTED.  The first
  * call on a device looks up that array's address and should come before any
  * stream capture.  All calls on a device share the array: calls that overlap
  * on the GPU race and must be serialised by the caller. */
@@ -194,7 +195,7 @@ moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const
                            float* f, float* p, float* l_aux, cudaStream_t stream);
 
 /* The whole layer forward: router, top-k, dispatch, expert FFNs, combine and
- * aux statistics, six kernel launches on `stream`.  `logits_in` as in
+ * aux statistics, five kernel launches on `stream`.  `logits_in` as in
  * moe_router_topk (NULL in normal use). */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
                          const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,

@@ -15,13 +15,16 @@ namespace moe {
 namespace {
 
 template <bool BF16>
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
+    constexpr int U = 4;               // 16-byte vectors per lane per expert row (x2 rows in flight)
+    constexpr int VEC = BF16 ? 8 : 4;  // elements per 16-byte vector
     const int warps_per_cta = blockDim.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t warp_g = (int64_t)blockIdx.x * warps_per_cta + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * warps_per_cta;
-    constexpr int VEC = BF16 ? 8 : 4;  // elements per 16-byte vector
     const int nvec = a.d / VEC;
+    const uint4* Y = reinterpret_cast<const uint4*>(a.y_perm);
+    uint4* O = reinterpret_cast<uint4*>(a.out);
     for (int64_t t = warp_g; t < a.T; t += nwarps) {
         int s_l = -1;
         float w_l = 0.f;
@@ -36,40 +39,61 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
             sj[j] = __shfl_sync(0xffffffffu, s_l, j);
             wj[j] = __shfl_sync(0xffffffffu, w_l, j);
         }
-        for (int v = lane; v < nvec; v += 32) {
-            float acc[VEC];
+        for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+            float acc[U][VEC];
 #pragma unroll
-            for (int q = 0; q < VEC; ++q) acc[q] = 0.f;
+            for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j >= a.k) break;
-                const int s = sj[j];
-                const float w = wj[j];
-                if (s < 0) continue;
-                const uint4 y = reinterpret_cast<const uint4*>(a.y_perm)[(int64_t)s * nvec + v];
-                if constexpr (BF16) {
-                    const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
+                for (int q = 0; q < VEC; ++q) acc[u][q] = 0.f;
+            // experts in pairs: 2*U loads in flight, then the FMAs in ascending j
+            for (int j = 0; j < a.k; j += 2) {
+                const int s0 = sj[j];
+                const int s1 = (j + 1 < a.k) ? sj[j + 1] : -1;
+                uint4 y0[U], y1[U];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[2 * q] = fmaf(w, bf16_lo(ys[q]), acc[2 * q]);
-                        acc[2 * q + 1] = fmaf(w, bf16_hi(ys[q]), acc[2 * q + 1]);
+                for (int u = 0; u < U; ++u) {
+                    const bool in = v0 + 32 * u < nvec;
+                    if (in && s0 >= 0) y0[u] = Y[(int64_t)s0 * nvec + v0 + 32 * u];
+                    if (in && s1 >= 0) y1[u] = Y[(int64_t)s1 * nvec + v0 + 32 * u];
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s = h ? s1 : s0;
+                    if (s < 0) continue;
+                    const float w = h ? wj[j + 1] : wj[j];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (v0 + 32 * u >= nvec) continue;
+                        const uint4 yv = h ? y1[u] : y0[u];
+                        if constexpr (BF16) {
+                            const uint32_t ys[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                acc[u][2 * q] = fmaf(w, bf16_lo(ys[q]), acc[u][2 * q]);
+                                acc[u][2 * q + 1] = fmaf(w, bf16_hi(ys[q]), acc[u][2 * q + 1]);
+                            }
+                        } else {
+                            acc[u][0] = fmaf(w, __uint_as_float(yv.x), acc[u][0]);
+                            acc[u][1] = fmaf(w, __uint_as_float(yv.y), acc[u][1]);
+                            acc[u][2] = fmaf(w, __uint_as_float(yv.z), acc[u][2]);
+                            acc[u][3] = fmaf(w, __uint_as_float(yv.w), acc[u][3]);
+                        }
                     }
-                } else {
-                    acc[0] = fmaf(w, __uint_as_float(y.x), acc[0]);
-                    acc[1] = fmaf(w, __uint_as_float(y.y), acc[1]);
-                    acc[2] = fmaf(w, __uint_as_float(y.z), acc[2]);
-                    acc[3] = fmaf(w, __uint_as_float(y.w), acc[3]);
                 }
             }
-            uint4 o;
-            if constexpr (BF16) {
-                o = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                               pack_bf16x2(acc[6], acc[7]));
-            } else {
-                o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                               __float_as_uint(acc[3]));
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (v0 + 32 * u >= nvec) continue;
+                uint4 o;
+                if constexpr (BF16) {
+                    o = make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
+                                   pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+                } else {
+                    o = make_uint4(__float_as_uint(acc[u][0]), __float_as_uint(acc[u][1]), __float_as_uint(acc[u][2]),
+                                   __float_as_uint(acc[u][3]));
+                }
+                O[t * nvec + v0 + 32 * u] = o;
             }
-            reinterpret_cast<uint4*>(a.out)[t * nvec + v] = o;
         }
     }
 }
@@ -132,7 +156,7 @@ __global__ void selftest_wait_kernel(DevStatus st) {
 
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
-    const int64_t blocks = min64((a.T + 7) / 8, (int64_t)sm_count() * 16);
+    const int64_t blocks = min64((a.T + 7) / 8, (int64_t)sm_count() * 8);
     if (bf16)
         combine_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(a);
     else

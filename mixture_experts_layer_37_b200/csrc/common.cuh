@@ -11,12 +11,15 @@ namespace moe {
 
 // Token chunk shared by the router (partial histograms / probability sums)
 // and the dispatch scatter (per-chunk rank bases).
-constexpr int kChunkTokens = 64;
+constexpr int kChunkTokens = 32;
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
 
 // Workspace status block: word 0 = error bits, word 1 = site of the first
-// wait that gave up, word 2 = a flag nothing ever sets (bounded-wait self-test).
+// wait that gave up, word 2 = a flag nothing ever sets (bounded-wait self-test),
+// word 4 = arrival counter of the router CTAs (the last one runs the scan; it
+// resets the counter to 0, and moe_workspace_init zeroes it).
+constexpr int kStatusCounterWord = 4;
 constexpr uint32_t kErrTimeout = 1u;
 enum WaitSite : uint32_t {
     SITE_NONE = 0,

@@ -9,11 +9,11 @@
 // Such a caller cannot provide the workspace that moe_dispatch needs for its
 // per-chunk histograms and rank bases.  This entry point keeps that scratch
 // in a fixed-size array in the library's own device memory instead
-// (`g_dispatch_scratch`, 512 KiB on every GPU that loads the library, held
+// (`g_dispatch_scratch`, 1 MiB on every GPU that loads the library, held
 // until the process exits).
 //
 // Limits and rules:
-//   - ceil(T / 64) * E must not exceed 65536 (for E = 64: T <= 65536 tokens);
+//   - ceil(T / 32) * E must not exceed 131072 (for E = 64: T <= 65536 tokens);
 //     larger shapes return MOE_ERR_UNSUPPORTED before anything is launched.
 //   - The first call on each device looks up the array's device address
 //     (cudaGetSymbolAddress) with that device current; make that first call
@@ -30,7 +30,7 @@
 
 namespace {
 
-constexpr int64_t kNoAllocMaxEntries = 65536;  // ceil(T/64) * E
+constexpr int64_t kNoAllocMaxEntries = 131072;  // ceil(T/32) * E
 constexpr int kMaxDevices = 64;
 
 // [0, kNoAllocMaxEntries): per-chunk expert histogram; [kNoAllocMaxEntries, 2x): per-chunk rank bases.
@@ -109,6 +109,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     xa.E = cfg->E;
     xa.k = cfg->k;
     xa.cap = (int)cap;
+    xa.nchunk = (int)nchunk;
     xa.row_bytes = (int)(cfg->d * (cfg->dtype == MOE_DT_BF16 ? 2 : 4));
     if (moe::launch_dispatch_scatter(xa, stream) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;

@@ -44,7 +44,9 @@ constexpr int kBStageBytes = 4 * kBBoxBytes;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;   // 48 KB
 constexpr int kTmemCols = 2 * BN_MMA;                      // two fp32 accumulators
 constexpr int kThreads = 192;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers + tables*/ + 1024 /*alignment*/;
+constexpr int kGroupM = 32;  // m-tiles per raster group
+constexpr int kBiasBytes = 4 * BN_MMA * 2;                 // one bf16 bias row per epilogue warp
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + 1024 /*alignment*/;
 
 enum { MODE_PLAIN = 0, MODE_SWIGLU = 1, MODE_GELU = 2 };
 
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* mt_prefix = reinterpret_cast<int*>(tmem_slot + 2);   // [E+1]
     int* s_off = mt_prefix + (kMaxExperts + 1);                // [E+1]
+    __nv_bfloat16* s_bias = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes + 1024);  // [4][256]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -139,12 +142,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kblocks = p.K / BK;
     const uint64_t tmo = p.st.timeout_ns;
 
+    // Tile order: expert by expert; inside an expert, groups of kGroupM
+    // m-tiles, and inside a group n-tile-major.  The CTAs running at the same
+    // time then share each weight tile among up to kGroupM of them and each
+    // activation tile among the group's n-tiles, which keeps the expert's
+    // working set in L2 even when its weights exceed it.
     auto decode = [&](int tile, int& e, int& row0, int& rows, int& nt) {
-        const int mt = tile / p.n_tiles;
-        nt = tile - mt * p.n_tiles;
         e = 0;
-        while (mt_prefix[e + 1] <= mt) ++e;
-        row0 = s_off[e] + (mt - mt_prefix[e]) * BM;
+        while (mt_prefix[e + 1] * p.n_tiles <= tile) ++e;
+        const int local = tile - mt_prefix[e] * p.n_tiles;
+        const int mt_e = mt_prefix[e + 1] - mt_prefix[e];
+        const int grp = local / (kGroupM * p.n_tiles);
+        const int gm = min(kGroupM, mt_e - grp * kGroupM);
+        const int r = local - grp * kGroupM * p.n_tiles;
+        nt = r / gm;
+        const int mt = grp * kGroupM + (r - nt * gm);
+        row0 = s_off[e] + mt * BM;
         rows = min(BM, s_off[e + 1] - row0);
     };
     auto give_up = [&](uint32_t site) {
@@ -288,6 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
+                // this tile's 256 bias values, staged once per tile in the warp's own row
+                __nv_bfloat16* wb = s_bias + (warp - 2) * BN_MMA;
+                if (p.bias != nullptr) {
+                    __syncwarp();
+                    const int col = n0 + 8 * lane;
+                    uint4 bv = make_uint4(0, 0, 0, 0);
+                    if (col < p.N) bv = *reinterpret_cast<const uint4*>(p.bias + (int64_t)e * p.N + col);
+                    reinterpret_cast<uint4*>(wb)[lane] = bv;
+                    __syncwarp();
+                }
                 for (int c = 0; c < BN_MMA; c += 16) {
                     uint32_t v[16];
                     tmem_ld_16(tbase + c, v);
@@ -297,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(v[i]);
                         if (p.bias != nullptr) {
-                            const __nv_bfloat16* b = p.bias + (int64_t)e * p.N + n0 + c;
+                            const __nv_bfloat16* b = wb + c;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) x[i] += __bfloat162float(b[i]);
                         }

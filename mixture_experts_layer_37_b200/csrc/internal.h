@@ -10,26 +10,10 @@
 
 namespace moe {
 
-struct RouterArgs {
-    const void* x;           // [T, d] act dtype
-    const void* w_router;    // [d, E] act dtype
-    const float* bias;       // [E] or null
-    const float* logits_in;  // [T, E] or null
-    int32_t* topk_idx;       // [T, k]
-    float* topk_w;           // [T, k]
-    float* logits_out;       // [T, E] or null
-    float* probs_out;        // [T, E] or null
-    int32_t* hist;           // [nchunk, E] per-chunk expert histogram
-    double* psum;            // [nchunk, E] per-chunk sum of probabilities
-    int64_t T;
-    int d, E, k;
-};
-cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
-
 struct ScanArgs {
-    const int32_t* hist;   // [nchunk, E]
-    const double* psum;    // [nchunk, E] or null (no aux stats)
-    int32_t* chunk_base;   // [nchunk, E] out
+    const int32_t* hist;   // [E, nchunk] per-chunk expert histogram
+    const double* psum;    // [E, nchunk] per-chunk probability sums, or null (no aux stats)
+    int32_t* chunk_base;   // [E, nchunk] out: assignments to e in earlier chunks
     int32_t* counts;       // [E] out
     int32_t* offsets;      // [E+1] out
     float* f;              // [E] out or null
@@ -39,19 +23,42 @@ struct ScanArgs {
     int nchunk, E, k, cap;
     float alpha;
 };
+
+struct RouterArgs {
+    const void* x;           // [T, d] act dtype
+    const void* w_router;    // [d, E] act dtype
+    const float* bias;       // [E] or null
+    const float* logits_in;  // [T, E] or null
+    int32_t* topk_idx;       // [T, k]
+    float* topk_w;           // [T, k]
+    float* logits_out;       // [T, E] or null
+    float* probs_out;        // [T, E] or null
+    int32_t* hist;           // [E, nchunk] per-chunk expert histogram
+    double* psum;            // [E, nchunk] per-chunk sum of probabilities
+    int64_t T;
+    int d, E, k, nchunk;
+    int tpc;                 // tokens per CTA (set by the launcher; multiple of the chunk)
+    // when fuse_scan != 0: the last CTA to finish (counted on `counter`) runs
+    // the dispatch scan and the aux statistics described by `scan`
+    int fuse_scan;
+    unsigned int* counter;
+    ScanArgs scan;
+};
+cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
+
 cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s);
 
 struct ScatterArgs {
     const int32_t* topk_idx;    // [T, k]
-    const int32_t* chunk_base;  // [nchunk, E]
+    const int32_t* chunk_base;  // [E, nchunk]
     const int32_t* offsets;     // [E+1]
     int32_t* slot;              // [T, k]
     int32_t* src_assign;        // [R_max]
     const void* x;              // [T, d]
     void* x_perm;               // [R_max, d]
     int64_t T;
-    int E, k, cap;
+    int E, k, cap, nchunk;
     int row_bytes;              // d * element size (multiple of 16)
 };
 cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);

@@ -133,37 +133,15 @@ moe_status_t check_weights(const moe_config_t* c, const moe_weights_t* w, bool n
         if (c->act == MOE_ACT_SWIGLU) {
             if (w->w_up == nullptr || !aligned16(w->w_up)) return MOE_ERR_INVALID_ARG;
         } else {
-            if (w->b1 == nullptr || w->b2 == nullptr) return MOE_ERR_INVALID_ARG;
+            if (w->b1 == nullptr || w->b2 == nullptr || !aligned16(w->b1) || !aligned16(w->b2))
+                return MOE_ERR_INVALID_ARG;
         }
     }
     return MOE_OK;
 }
 
-moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_router, const float* bias,
-                        const float* logits_in, int32_t* idx, float* w, float* logits_out, float* probs_out,
-                        void* ws, const Plan& pl, cudaStream_t s) {
-    RouterArgs a;
-    a.x = x;
-    a.w_router = w_router;
-    a.bias = bias;
-    a.logits_in = logits_in;
-    a.topk_idx = idx;
-    a.topk_w = w;
-    a.logits_out = logits_out;
-    a.probs_out = probs_out;
-    a.hist = reinterpret_cast<int32_t*>(at(ws, pl.hist));
-    a.psum = reinterpret_cast<double*>(at(ws, pl.psum));
-    a.T = c->T;
-    a.d = c->d;
-    a.E = c->E;
-    a.k = c->k;
-    return from_cuda(launch_router(a, c->dtype == MOE_DT_BF16, s));
-}
-
-moe_status_t run_scan_scatter(const moe_config_t* c, const void* x, const int32_t* idx, int32_t* counts,
-                              int32_t* offsets, int32_t* slot, int32_t* src_assign, void* x_perm, float* f, float* p,
-                              float* l_aux, bool with_stats, void* ws, const Plan& pl, cudaStream_t s,
-                              cudaEvent_t between = nullptr) {
+ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, float* f, float* p, float* l_aux,
+                   bool with_stats, void* ws, const Plan& pl) {
     ScanArgs sa;
     sa.hist = reinterpret_cast<const int32_t*>(at(ws, pl.hist));
     sa.psum = with_stats ? reinterpret_cast<const double*>(at(ws, pl.psum)) : nullptr;
@@ -179,13 +157,40 @@ moe_status_t run_scan_scatter(const moe_config_t* c, const void* x, const int32_
     sa.k = c->k;
     sa.cap = (int)capacity_used(c);
     sa.alpha = c->aux_alpha;
-    cudaError_t e = launch_dispatch_scan(sa, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (sa.nchunk == 0) return MOE_OK;
-    if (between != nullptr && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return sa;
+}
+
+// Router; with `fused` set, its last CTA also runs the scan described by `sa`.
+moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_router, const float* bias,
+                        const float* logits_in, int32_t* idx, float* w, float* logits_out, float* probs_out,
+                        void* ws, const Plan& pl, cudaStream_t s, const ScanArgs* fused = nullptr) {
+    RouterArgs a;
+    a.x = x;
+    a.w_router = w_router;
+    a.bias = bias;
+    a.logits_in = logits_in;
+    a.topk_idx = idx;
+    a.topk_w = w;
+    a.logits_out = logits_out;
+    a.probs_out = probs_out;
+    a.hist = reinterpret_cast<int32_t*>(at(ws, pl.hist));
+    a.psum = reinterpret_cast<double*>(at(ws, pl.psum));
+    a.T = c->T;
+    a.d = c->d;
+    a.E = c->E;
+    a.k = c->k;
+    a.nchunk = pl.nchunk;
+    a.fuse_scan = fused != nullptr ? 1 : 0;
+    a.counter = static_cast<unsigned int*>(ws) + kStatusCounterWord;
+    if (fused != nullptr) a.scan = *fused;
+    return from_cuda(launch_router(a, c->dtype == MOE_DT_BF16, s));
+}
+
+moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* idx, const int32_t* offsets,
+                         int32_t* slot, int32_t* src_assign, void* x_perm, void* ws, const Plan& pl, cudaStream_t s) {
     ScatterArgs xa;
     xa.topk_idx = idx;
-    xa.chunk_base = sa.chunk_base;
+    xa.chunk_base = reinterpret_cast<const int32_t*>(at(ws, pl.base));
     xa.offsets = offsets;
     xa.slot = slot;
     xa.src_assign = src_assign;
@@ -194,7 +199,8 @@ moe_status_t run_scan_scatter(const moe_config_t* c, const void* x, const int32_
     xa.T = c->T;
     xa.E = c->E;
     xa.k = c->k;
-    xa.cap = sa.cap;
+    xa.cap = (int)capacity_used(c);
+    xa.nchunk = pl.nchunk;
     xa.row_bytes = (int)(c->d * elem_size(c));
     return from_cuda(launch_dispatch_scatter(xa, s));
 }
@@ -308,8 +314,9 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
     if (launch_dispatch_hist(topk_idx, reinterpret_cast<int32_t*>(at(ws, pl.hist)), cfg->T, cfg->E, cfg->k, stream) !=
         cudaSuccess)
         return MOE_ERR_CUDA;
-    return run_scan_scatter(cfg, x, topk_idx, counts, offsets, slot, src_assign, x_perm, nullptr, nullptr, nullptr,
-                            false, ws, pl, stream);
+    const ScanArgs sa = scan_args(cfg, counts, offsets, nullptr, nullptr, nullptr, false, ws, pl);
+    if (launch_dispatch_scan(sa, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    return run_scatter(cfg, x, topk_idx, offsets, slot, src_assign, x_perm, ws, pl, stream);
 }
 
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_perm,
@@ -362,19 +369,22 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
     int n = 0;
     auto mark = [&]() -> bool { return ev == nullptr || cudaEventRecord(ev[n++], stream) == cudaSuccess; };
-    if (cfg->T > 0) {
+    const ScanArgs sa = scan_args(cfg, o->counts, o->offsets, o->f, o->p, o->l_aux, true, ws, pl);
+    if (cfg->T == 0) {
+        // nothing to route: one launch writes the zero counts, offsets and statistics
         if (!mark()) return MOE_ERR_CUDA;
-        st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
-                        o->logits_out, o->probs_out, ws, pl, stream);
-        if (st != MOE_OK) return st;
+        if (launch_dispatch_scan(sa, stream) != cudaSuccess) return MOE_ERR_CUDA;
+        return mark() ? MOE_OK : MOE_ERR_CUDA;
     }
     void* x_perm = at(ws, pl.xperm);
     void* y_perm = at(ws, pl.yperm);
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_scan_scatter(cfg, x, o->topk_idx, o->counts, o->offsets, o->slot, o->src_assign, x_perm, o->f, o->p,
-                          o->l_aux, true, ws, pl, stream, (ev && cfg->T > 0) ? ev[n++] : nullptr);
+    st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
+                    o->logits_out, o->probs_out, ws, pl, stream, &sa);
     if (st != MOE_OK) return st;
-    if (cfg->T == 0) return mark() ? MOE_OK : MOE_ERR_CUDA;
+    if (!mark()) return MOE_ERR_CUDA;
+    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, x_perm, ws, pl, stream);
+    if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
     st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr);
     if (st != MOE_OK) return st;
@@ -443,7 +453,7 @@ moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint32_t timeo
 int32_t moe_forward_launch_count(const moe_config_t* cfg) {
     if (check_config(cfg) != MOE_OK) return 0;
     if (cfg->T == 0) return 1;
-    return 6;
+    return 5;
 }
 
 }  // extern "C"

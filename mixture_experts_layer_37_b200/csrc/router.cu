@@ -1,33 +1,41 @@
 // Router kernel: logits = x . W_r (+ bias), fp32 softmax over all experts,
 // top-k on the logits (lower id first on ties), renormalised top-k weights,
-// and per-chunk partial statistics (expert histogram, sum of probabilities)
-// for the dispatch scan and the load-balance loss.
+// and per-chunk partial statistics (expert histogram, sum of probabilities);
+// in moe_forward the last CTA to finish also runs the dispatch scan and the
+// load-balance statistics.
 //
 // Method: "MoE: gating, experts, load balancing, capacity factor"
 // (dpshk.com/news/6005940) §2.1 (score = x . W_r, softmax) and §3.1 (top-k);
 // "Llama-MoE架构解析" (coreui.cn/article/2610641) §3.1 (softmax -> top-k ->
 // divide by the sum of the k weights).
 //
-// One CTA per chunk of kChunkTokens tokens.  bf16: each warp computes 16
-// tokens x E logits with mma.sync m16n8k16 (fp32 accumulate).  x is streamed
-// once from HBM with 16-byte loads; the (small) router weight is staged in
-// shared memory, transposed, in K slabs.  The 32 reduction indices of one
-// step are assigned to MMA fragment positions so that every thread loads 16
-// contiguous bytes of x (the same assignment is used for W_r, so the product
-// is unchanged).  f32: one thread per token, fp32 FMA.
+// bf16: one CTA of 8 warps per `tpc` tokens (32, 64 or 128: enough CTAs to
+// fill the GPU, and enough tokens per CTA that re-reading the router weight
+// per CTA stays small next to the x stream).  The warps form tpc/16 token
+// groups x 128/tpc K-splits.  Each warp streams its x rows once from HBM with
+// 16-byte loads, four 32-column blocks (8 loads per lane) in flight per batch
+// and two CTAs per SM, and multiplies on the tensor cores with mma.sync m16n8k16 (bf16 in,
+// fp32 accumulate).  The router weight [d, E] is copied into shared memory as
+// it lies in HBM (16-byte rows per 8 experts) in K slabs, and ldmatrix.trans
+// turns it into MMA B fragments.  Inside each MMA the 32 reduction indices of
+// a step are assigned so that a thread's A fragment is 16 contiguous bytes of
+// x; the ldmatrix row addresses apply the same assignment to W_r, so the
+// product is unchanged.  Slab rows are stored rotated within 32-row blocks and
+// padded to an odd number of 16-byte units, so the eight rows of every
+// ldmatrix phase fall in eight distinct bank groups.  K-split partial sums
+// are added in a fixed order.  f32: one thread per token, fp32 FMA.
 #include <math.h>
 
-#include "internal.h"
+#include "scan.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 128;          // 4 warps x 16 tokens = kChunkTokens
-constexpr int kSlabK = 512;            // K slab of W_r held in shared memory (bf16)
-constexpr int kSlabPad = 32;           // row padding (elements): conflict-free 16-byte reads
-constexpr int kSlabStride = kSlabK + kSlabPad;
+constexpr int kThreads = 256;
 constexpr int kLStride = kMaxExperts + 1;
-static_assert(kChunkTokens == 64, "router tiling assumes 64-token chunks");
+constexpr int kSlabBytes = 64 * 1024;
+constexpr int kMaxTpc = 128;
+constexpr int kBatch = 4;  // 32-column blocks of x loaded per batch
 
 __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
     uint4 v;
@@ -35,6 +43,12 @@ __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -46,15 +60,23 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Softmax / top-k / renormalisation / partial statistics for the chunk whose
-// logits sit in sL[token][e].  Called by all threads of the CTA.
+// Row position of slab row kk: rotated inside its 32-row block.
+__device__ __forceinline__ int slab_phys_row(int kk) {
+    const int a = (kk >> 3) & 3, b = kk & 7;
+    return (kk & ~31) + 8 * a + ((b + 2 * a) & 7);
+}
+
+// Softmax / top-k / renormalisation / per-chunk partial statistics for the
+// CTA's tokens, whose logits sit in sL[token][e]; then, when fusing, the last
+// CTA to arrive runs the dispatch scan.  All threads of the CTA call it.
 __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool add_bias) {
     const int tid = threadIdx.x;
     const int E = a.E, k = a.k;
-    const int chunk = blockIdx.x;
-    const int64_t t0 = (int64_t)chunk * kChunkTokens;
-    const int ntok = (int)min64(kChunkTokens, a.T - t0);
-    if (tid < E) sHist[tid] = 0;
+    const int64_t t0 = (int64_t)blockIdx.x * a.tpc;
+    const int ntok = (int)min64(a.tpc, a.T - t0);
+    const int nchk = (ntok + kChunkTokens - 1) / kChunkTokens;
+    const int chunk0 = (int)(t0 / kChunkTokens);
+    for (int i = tid; i < nchk * kMaxExperts; i += blockDim.x) sHist[i] = 0;
     __syncthreads();
     if (tid < ntok) {
         const int64_t t = t0 + tid;
@@ -77,7 +99,10 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
             for (int e = 0; e < E; ++e) {
                 if ((chosen >> e) & 1ull) continue;
                 const float v = row[e];
-                if (best < 0 || v > bv) { best = e; bv = v; }
+                if (best < 0 || v > bv) {
+                    best = e;
+                    bv = v;
+                }
             }
             chosen |= 1ull << best;
             sel_idx[j] = best;
@@ -97,24 +122,41 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
         }
         float ps = 0.f;
         for (int j = 0; j < k; ++j) ps += row[sel_idx[j]];
+        int* hrow = sHist + (tid / kChunkTokens) * kMaxExperts;
         for (int j = 0; j < k; ++j) {
             a.topk_idx[t * k + j] = sel_idx[j];
             a.topk_w[t * k + j] = row[sel_idx[j]] / ps;
-            atomicAdd(&sHist[sel_idx[j]], 1);
+            atomicAdd(&hrow[sel_idx[j]], 1);
         }
     }
     __syncthreads();
-    if (tid < E) {
+    for (int i = tid; i < nchk * E; i += blockDim.x) {
+        const int cl = i / E, e = i - cl * E;
+        const int i0 = cl * kChunkTokens, i1 = min(ntok, i0 + kChunkTokens);
         double acc = 0.0;
-        for (int i = 0; i < ntok; ++i) acc += (double)sL[i * kLStride + tid];
-        a.psum[(int64_t)chunk * E + tid] = acc;
-        a.hist[(int64_t)chunk * E + tid] = sHist[tid];
+        for (int r = i0; r < i1; ++r) acc += (double)sL[r * kLStride + e];
+        a.psum[(int64_t)e * a.nchunk + chunk0 + cl] = acc;
+        a.hist[(int64_t)e * a.nchunk + chunk0 + cl] = sHist[cl * kMaxExperts + e];
     }
+    if (!a.fuse_scan) return;
+    // last-CTA-done: the CTA that completes the arrival count runs the scan on
+    // everyone's partials (fences order the partial stores before the count)
+    __shared__ int sLast;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sLast = (atomicAdd(a.counter, 1u) == (unsigned)gridDim.x - 1u) ? 1 : 0;
+    __syncthreads();
+    if (!sLast) return;
+    __threadfence();
+    __shared__ int sCount[kMaxExperts];
+    __shared__ double sP[kMaxExperts];
+    scan_block(a.scan, sCount, sP);
+    if (tid == 0) *a.counter = 0u;
 }
 
 __device__ void load_logits_in(const RouterArgs& a, float* sL) {
-    const int64_t t0 = (int64_t)blockIdx.x * kChunkTokens;
-    const int ntok = (int)min64(kChunkTokens, a.T - t0);
+    const int64_t t0 = (int64_t)blockIdx.x * a.tpc;
+    const int ntok = (int)min64(a.tpc, a.T - t0);
     for (int i = threadIdx.x; i < ntok * a.E; i += blockDim.x) {
         const int tok = i / a.E, e = i - tok * a.E;
         sL[tok * kLStride + e] = a.logits_in[(t0 + tok) * a.E + e];
@@ -122,12 +164,36 @@ __device__ void load_logits_in(const RouterArgs& a, float* sL) {
     __syncthreads();
 }
 
+template <int NT>
+struct SlabGeom {
+    static constexpr int kUnits = (NT & 1) ? NT : NT + 1;   // odd row pitch in 16-byte units
+    static constexpr int kPitch = 16 * kUnits;
+    static constexpr int kRows = (kSlabBytes / kPitch) / 128 * 128;
+    static constexpr int kPartBytes = 128 * 8 * NT * 4;     // nsplit * tpc = 128 rows of EP floats
+};
+
+// Bytes of the shared region that holds the weight slab, and after the K
+// loop the K-split partial logits.
+template <int NT>
+__host__ __device__ __forceinline__ int union_bytes_for(int d) {
+    const int rows = SlabGeom<NT>::kRows < d ? SlabGeom<NT>::kRows : d;
+    const int slab = (rows * SlabGeom<NT>::kPitch + 127) & ~127;
+    return slab > SlabGeom<NT>::kPartBytes ? slab : SlabGeom<NT>::kPartBytes;
+}
+
+__host__ __device__ __forceinline__ int tail_bytes_for(int tpc) {
+    return tpc * kLStride * 4 + (kMaxTpc / kChunkTokens) * kMaxExperts * 4;
+}
+
 template <int NT>  // experts padded to 8*NT
-__global__ void __launch_bounds__(kThreads) router_bf16_kernel(RouterArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    float* sL = reinterpret_cast<float*>(smem);                                       // [64][65]
-    int* sHist = reinterpret_cast<int*>(smem + kChunkTokens * kLStride * 4);          // [64]
-    __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem + kChunkTokens * kLStride * 4 + 256);  // [8NT][stride]
+__global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) {
+    using G = SlabGeom<NT>;
+    constexpr int EP = 8 * NT;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t* sW = smem;                                                // slab, then partials
+    float* sPart = reinterpret_cast<float*>(smem);                     // [nsplit][tpc][EP]
+    float* sL = reinterpret_cast<float*>(smem + union_bytes_for<NT>(a.d));  // [tpc][65]
+    int* sHist = reinterpret_cast<int*>(sL + a.tpc * kLStride);        // [tpc/32][64]
 
     if (a.logits_in) {
         load_logits_in(a, sL);
@@ -136,91 +202,125 @@ __global__ void __launch_bounds__(kThreads) router_bf16_kernel(RouterArgs a) {
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
+    const int ngroups = a.tpc / 16, nsplit = 8 / ngroups;
+    const int tg = warp % ngroups, ksplit = warp / ngroups;
     const int E = a.E, d = a.d;
-    const int64_t t0 = (int64_t)blockIdx.x * kChunkTokens;
-    const int64_t r0 = t0 + warp * 16 + g, r1 = r0 + 8;
+    const int64_t t0 = (int64_t)blockIdx.x * a.tpc;
+    const int64_t r0 = t0 + tg * 16 + g, r1 = r0 + 8;
     const bool v0 = r0 < a.T, v1 = r1 < a.T;
     const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(a.x);
     const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.w_router);
-    const __nv_bfloat16* x0 = X + (v0 ? r0 : 0) * (int64_t)d;
-    const __nv_bfloat16* x1 = X + (v1 ? r1 : 0) * (int64_t)d;
+    const __nv_bfloat16* x0 = X + (v0 ? r0 : 0) * (int64_t)d + 8 * c;
+    const __nv_bfloat16* x1 = X + (v1 ? r1 : 0) * (int64_t)d + 8 * c;
+    // ldmatrix lane j = lane/8 (fragment), r = lane%8 (matrix row): logical
+    // k = 8*(r/2) + 2j + (r%2) of the 32-row block, stored at its rotated row.
+    const int lj = lane >> 3, lr = lane & 7;
+    const int la = lr >> 1, lb = 2 * lj + (lr & 1);
+    const uint32_t lds_base = smem_u32(sW) + (uint32_t)((8 * la + ((lb + 2 * la) & 7)) * G::kPitch);
 
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
-    const __nv_bfloat16 zero = __float2bfloat16(0.f);
-    for (int k0 = 0; k0 < d; k0 += kSlabK) {
-        const int ks = min(kSlabK, d - k0);  // multiple of 64
+    const bool vec_rows = (E & 7) == 0;
+    for (int k0 = 0; k0 < d; k0 += G::kRows) {
+        const int ks = min(G::kRows, d - k0);  // multiple of 64
         __syncthreads();
-        // stage W_r[k0:k0+ks, :] transposed: sW[e][kk]
-        if ((E & 7) == 0) {
-            for (int kk = tid; kk < ks; kk += kThreads) {
-                const uint4* src = reinterpret_cast<const uint4*>(W + (int64_t)(k0 + kk) * E);
-                for (int e8 = 0; e8 < E / 8; ++e8) {
-                    const uint4 v = src[e8];
-                    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+        // stage W_r[k0 : k0+ks, :] (16-byte units, batched loads)
+        const int nunits = ks * NT;
+        for (int i0 = tid; i0 < nunits; i0 += kThreads * 8) {
+            uint4 v[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) sW[(e8 * 8 + q) * kSlabStride + kk] = h[q];
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * kThreads;
+                if (i >= nunits) break;
+                const int kk = i / NT, q = i - kk * NT;
+                if (vec_rows) {
+                    v[u] = *reinterpret_cast<const uint4*>(W + (int64_t)(k0 + kk) * E + 8 * q);
+                } else {
+                    __nv_bfloat16 h[8];
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const int e = 8 * q + w;
+                        h[w] = e < E ? W[(int64_t)(k0 + kk) * E + e] : __float2bfloat16(0.f);
+                    }
+                    v[u] = *reinterpret_cast<const uint4*>(h);
                 }
-                for (int e = E; e < 8 * NT; ++e) sW[e * kSlabStride + kk] = zero;
             }
-        } else {
-            for (int kk = tid; kk < ks; kk += kThreads) {
-                for (int e = 0; e < 8 * NT; ++e)
-                    sW[e * kSlabStride + kk] = e < E ? W[(int64_t)(k0 + kk) * E + e] : zero;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * kThreads;
+                if (i >= nunits) break;
+                const int kk = i / NT, q = i - kk * NT;
+                *reinterpret_cast<uint4*>(sW + slab_phys_row(kk) * G::kPitch + 16 * q) = v[u];
             }
         }
         __syncthreads();
-        for (int kk = 0; kk < ks; kk += 64) {
-            uint4 xa[2], xb[2];
+        // this warp's 32-row blocks of the slab: ksplit, ksplit + nsplit, ...
+        const int nblk = ks / 32;
+        for (int b0 = ksplit; b0 < nblk; b0 += nsplit * kBatch) {
+            uint4 xa[kBatch], xb[kBatch];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                xa[u] = v0 ? ldg_stream_128(x0 + k0 + kk + 32 * u + 8 * c) : make_uint4(0, 0, 0, 0);
-                xb[u] = v1 ? ldg_stream_128(x1 + k0 + kk + 32 * u + 8 * c) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < kBatch; ++u) {
+                const int blk = b0 + u * nsplit;
+                const int kx = k0 + 32 * blk;
+                xa[u] = (blk < nblk && v0) ? ldg_stream_128(x0 + kx) : make_uint4(0, 0, 0, 0);
+                xb[u] = (blk < nblk && v1) ? ldg_stream_128(x1 + kx) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < kBatch; ++u) {
+                const int blk = b0 + u * nsplit;
+                if (blk >= nblk) break;
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
-                    const uint4 bw = *reinterpret_cast<const uint4*>(sW + (n * 8 + g) * kSlabStride + kk + 32 * u + 8 * c);
-                    mma_bf16_16816(acc[n], xa[u].x, xb[u].x, xa[u].y, xb[u].y, bw.x, bw.y);
-                    mma_bf16_16816(acc[n], xa[u].z, xb[u].z, xa[u].w, xb[u].w, bw.z, bw.w);
+                    uint32_t b0r, b1r, b2r, b3r;
+                    ldsm_x4_trans(lds_base + (uint32_t)(32 * blk * G::kPitch + 16 * n), b0r, b1r, b2r, b3r);
+                    mma_bf16_16816(acc[n], xa[u].x, xb[u].x, xa[u].y, xb[u].y, b0r, b1r);
+                    mma_bf16_16816(acc[n], xa[u].z, xb[u].z, xa[u].w, xb[u].w, b2r, b3r);
                 }
             }
         }
     }
-    // accumulators -> sL[token][e]
+    __syncthreads();  // the slab region is reused for the partials
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int e0 = n * 8 + 2 * c;
-        float* ra = sL + (warp * 16 + g) * kLStride;
-        float* rb = sL + (warp * 16 + g + 8) * kLStride;
-        ra[e0] = acc[n][0];
-        ra[e0 + 1] = acc[n][1];
-        rb[e0] = acc[n][2];
-        rb[e0 + 1] = acc[n][3];
+        float* pa = sPart + (ksplit * a.tpc + tg * 16 + g) * EP;
+        float* pb = pa + 8 * EP;
+        pa[e0] = acc[n][0];
+        pa[e0 + 1] = acc[n][1];
+        pb[e0] = acc[n][2];
+        pb[e0 + 1] = acc[n][3];
+    }
+    __syncthreads();
+    const int split_stride = a.tpc * EP;
+    for (int i = tid; i < a.tpc * E; i += kThreads) {
+        const int tok = i / E, e = i - tok * E;
+        const float* p = sPart + tok * EP + e;
+        float v = p[0];
+        for (int s = 1; s < nsplit; ++s) v += p[s * split_stride];
+        sL[tok * kLStride + e] = v;
     }
     __syncthreads();
     router_finish(a, sL, sHist, true);
 }
 
-template <int EP>  // experts padded to EP (8 or 64)
+template <int EP>  // experts padded to EP (8 or 64); tpc = 32
 __global__ void __launch_bounds__(kThreads) router_f32_kernel(RouterArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    float* sL = reinterpret_cast<float*>(smem);
-    int* sHist = reinterpret_cast<int*>(smem + kChunkTokens * kLStride * 4);
-    float* sW = reinterpret_cast<float*>(smem + kChunkTokens * kLStride * 4 + 256);  // [slab][EP]
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* sW = reinterpret_cast<float*>(smem);                                // [slab][EP]
+    float* sL = reinterpret_cast<float*>(smem + kSlabBytes);                   // [32][65]
+    int* sHist = reinterpret_cast<int*>(sL + kChunkTokens * kLStride);
     if (a.logits_in) {
         load_logits_in(a, sL);
         router_finish(a, sL, sHist, false);
         return;
     }
-    constexpr int kSlab = 8192 / EP;  // 32 KB of fp32 weights per slab
+    constexpr int kSlab = kSlabBytes / 4 / EP;
     const int tid = threadIdx.x;
     const int E = a.E, d = a.d;
-    const int64_t t = (int64_t)blockIdx.x * kChunkTokens + tid;
-    const bool valid = tid < kChunkTokens && t < a.T;
+    const int64_t t = (int64_t)blockIdx.x * a.tpc + tid;
+    const bool valid = tid < a.tpc && t < a.T;
     const float* X = static_cast<const float*>(a.x);
     const float* W = static_cast<const float*>(a.w_router);
     float acc[EP];
@@ -252,43 +352,70 @@ __global__ void __launch_bounds__(kThreads) router_f32_kernel(RouterArgs a) {
     router_finish(a, sL, sHist, true);
 }
 
+// Tokens per CTA: at least 4E (router weight re-read per CTA <= 1/4 of its
+// x bytes), at most 128, and small enough to give >= ~1 CTA per SM.
+int pick_tpc(int64_t T, int E) {
+    int tpc = 32;
+    while (tpc < 4 * E && tpc < kMaxTpc) tpc *= 2;
+    const int64_t sms = sm_count();
+    while (tpc > 32 && (T + tpc - 1) / tpc < sms) tpc /= 2;
+    return tpc;
+}
+
 template <int NT>
-cudaError_t launch_bf16_nt(const RouterArgs& a, int nchunk, cudaStream_t s) {
-    const size_t smem = kChunkTokens * kLStride * 4 + 256 + (size_t)8 * NT * kSlabStride * 2;
-    cudaError_t err = cudaFuncSetAttribute(router_bf16_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    router_bf16_kernel<NT><<<nchunk, kThreads, smem, s>>>(a);
+cudaError_t launch_bf16_nt(RouterArgs a, cudaStream_t s) {
+    a.tpc = pick_tpc(a.T, a.E);
+    const size_t smem = (size_t)union_bytes_for<NT>(a.d) + tail_bytes_for(a.tpc);
+    const size_t smem_max = (size_t)union_bytes_for<NT>(1 << 30) + tail_bytes_for(kMaxTpc);
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr[dev]) {
+        cudaError_t err =
+            cudaFuncSetAttribute(router_bf16_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+        if (err != cudaSuccess) return err;
+        if (dev < 64) attr[dev] = true;
+    }
+    const int grid = (int)((a.T + a.tpc - 1) / a.tpc);
+    router_bf16_kernel<NT><<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
 template <int EP>
-cudaError_t launch_f32_ep(const RouterArgs& a, int nchunk, cudaStream_t s) {
-    const size_t smem = kChunkTokens * kLStride * 4 + 256 + (size_t)8192 * 4;
-    cudaError_t err = cudaFuncSetAttribute(router_f32_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    router_f32_kernel<EP><<<nchunk, kThreads, smem, s>>>(a);
+cudaError_t launch_f32_ep(RouterArgs a, cudaStream_t s) {
+    a.tpc = kChunkTokens;
+    const size_t smem = kSlabBytes + tail_bytes_for(a.tpc);
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr[dev]) {
+        cudaError_t err = cudaFuncSetAttribute(router_f32_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        if (dev < 64) attr[dev] = true;
+    }
+    const int grid = (int)((a.T + a.tpc - 1) / a.tpc);
+    router_f32_kernel<EP><<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s) {
-    const int nchunk = (int)((a.T + kChunkTokens - 1) / kChunkTokens);
-    if (nchunk == 0) return cudaSuccess;
+    if (a.T == 0) return cudaSuccess;
     if (bf16) {
         switch ((a.E + 7) / 8) {
-            case 1: return launch_bf16_nt<1>(a, nchunk, s);
-            case 2: return launch_bf16_nt<2>(a, nchunk, s);
-            case 3: return launch_bf16_nt<3>(a, nchunk, s);
-            case 4: return launch_bf16_nt<4>(a, nchunk, s);
-            case 5: return launch_bf16_nt<5>(a, nchunk, s);
-            case 6: return launch_bf16_nt<6>(a, nchunk, s);
-            case 7: return launch_bf16_nt<7>(a, nchunk, s);
-            default: return launch_bf16_nt<8>(a, nchunk, s);
+            case 1: return launch_bf16_nt<1>(a, s);
+            case 2: return launch_bf16_nt<2>(a, s);
+            case 3: return launch_bf16_nt<3>(a, s);
+            case 4: return launch_bf16_nt<4>(a, s);
+            case 5: return launch_bf16_nt<5>(a, s);
+            case 6: return launch_bf16_nt<6>(a, s);
+            case 7: return launch_bf16_nt<7>(a, s);
+            default: return launch_bf16_nt<8>(a, s);
         }
     }
-    if (a.E <= 8) return launch_f32_ep<8>(a, nchunk, s);
-    return launch_f32_ep<64>(a, nchunk, s);
+    if (a.E <= 8) return launch_f32_ep<8>(a, s);
+    return launch_f32_ep<64>(a, s);
 }
 
 }  // namespace moe
