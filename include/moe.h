@@ -201,6 +201,34 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, 
                          const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
+/* ---- Data-parallel sharding of one logical batch ----------------------
+ * One batch of T_global tokens split in contiguous slices over `world` ranks
+ * (rank r holds its slice as a batch of cfg->T tokens, slices in rank order),
+ * with the capacity, the drop order and the load-balance statistics of the
+ * WHOLE batch: under data parallelism the per-expert token counts are summed
+ * over replicas before the load-balance loss ("Hand-building a LLaMA4-MoE"
+ * §3.1), and the capacity cut then drops in the batch's token order.  Results
+ * equal a single moe_forward over the whole batch (row indices local).
+ *   1. moe_dp_route on every rank: router and top-k of the slice; writes the
+ *      slice's per-expert counts local_counts [E] (int32, device) and
+ *      probability sums local_psum [E] (float64, device).
+ *   2. the caller all-gathers them in rank order into all_counts [world, E]
+ *      and all_psum [world, E] (device), e.g. with NCCL.
+ *   3. moe_dp_finish on every rank: capacity left for the slice, dispatch,
+ *      expert FFNs, combine; outputs->counts, f, p, l_aux are the whole
+ *      batch's (identical on every rank).
+ * Both calls use the same workspace of moe_dp_workspace_size bytes; outputs
+ * src_assign and the sorted-row buffers hold up to moe_dp_max_rows rows. */
+moe_status_t moe_dp_workspace_size(const moe_config_t* cfg, int64_t T_global, size_t* bytes);
+moe_status_t moe_dp_max_rows(const moe_config_t* cfg, int64_t T_global, int64_t* rows);
+moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_weights_t* weights, const void* x,
+                          const float* logits_in, moe_outputs_t* outputs, int32_t* local_counts,
+                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream);
+moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
+                           const double* all_psum, int32_t world, int32_t rank, const moe_weights_t* weights,
+                           const void* x, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
+                           cudaStream_t stream);
+
 /* moe_forward, recording stage_events[i] on `stream` just before kernel
  * launch i and stage_events[n] after the last launch, n =
  * moe_forward_launch_count(cfg) (stage_events: caller-created CUDA events,

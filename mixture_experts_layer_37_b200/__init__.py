@@ -98,7 +98,8 @@ EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_wo
                     "moe_router_topk", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_aux_stats",
                     "moe_forward", "moe_forward_hostio", "moe_check_device_status", "moe_set_wait_timeout_ms",
                     "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled",
-                    "moe_dispatch_noalloc")
+                    "moe_dispatch_noalloc", "moe_dp_workspace_size", "moe_dp_max_rows", "moe_dp_route",
+                    "moe_dp_finish")
 
 
 # ---------------------------------------------------------------- config
@@ -327,3 +328,50 @@ def moe_dispatch_noalloc(cfg: MoEConfig, x, topk_idx, counts, offsets, slot, src
     f.restype = ctypes.c_int
     _check(f(ctypes.byref(cfg.c()), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(slot),
              _ptr(src_assign), _ptr(x_perm), _stream(stream)), "moe_dispatch_noalloc")
+
+
+# ---------------------------------------------------------------- data-parallel shards of one batch
+def moe_dp_workspace_size(cfg: MoEConfig, T_global: int) -> int:
+    L = lib()
+    f = L.moe_dp_workspace_size
+    f.argtypes = [_CFG, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]
+    f.restype = ctypes.c_int
+    v = ctypes.c_size_t()
+    _check(f(ctypes.byref(cfg.c()), int(T_global), ctypes.byref(v)), "moe_dp_workspace_size")
+    return v.value
+
+
+def moe_dp_max_rows(cfg: MoEConfig, T_global: int) -> int:
+    L = lib()
+    f = L.moe_dp_max_rows
+    f.argtypes = [_CFG, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+    f.restype = ctypes.c_int
+    v = ctypes.c_int64()
+    _check(f(ctypes.byref(cfg.c()), int(T_global), ctypes.byref(v)), "moe_dp_max_rows")
+    return v.value
+
+
+def moe_dp_route(cfg: MoEConfig, T_global: int, weights: dict, x, outputs: dict, local_counts, local_psum,
+                 ws: Workspace, logits_in=None, stream=None) -> None:
+    L = lib()
+    f = L.moe_dp_route
+    f.argtypes = [_CFG, ctypes.c_int64, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P, _P, _P,
+                  ctypes.c_size_t, _P]
+    f.restype = ctypes.c_int
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), ctypes.byref(wc), _ptr(x), _ptr(logits_in), ctypes.byref(oc),
+             _ptr(local_counts), _ptr(local_psum), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_route")
+
+
+def moe_dp_finish(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: int, rank: int, weights: dict, x,
+                  outputs: dict, ws: Workspace, stream=None) -> None:
+    L = lib()
+    f = L.moe_dp_finish
+    f.argtypes = [_CFG, ctypes.c_int64, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P,
+                  ctypes.POINTER(MoEOutputsC), _P, ctypes.c_size_t, _P]
+    f.restype = ctypes.c_int
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank),
+             ctypes.byref(wc), _ptr(x), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_finish")

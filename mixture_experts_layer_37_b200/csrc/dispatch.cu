@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
     int s = -1;
     if (e >= 0) {
         const int rank = sWarpBase[warp][e] + lrank;
-        if (rank < a.cap) {
+        const int cap = a.cap_e != nullptr ? a.cap_e[e] : a.cap;
+        if (rank < cap) {
             s = a.offsets[e] + rank;
             a.src_assign[s] = (int32_t)(a_base + tid);
         }
@@ -120,7 +121,56 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
     }
 }
 
+// One CTA: data-parallel shard preparation (see DpPrepareArgs).  The
+// assignment rank of this rank's tokens in the whole batch is the number of
+// assignments to the same expert on lower ranks plus the local rank, so this
+// rank may keep max(0, cap - base_e) more rows of expert e.  Sums over ranks
+// run in rank order.
+__global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
+    __shared__ int sKept[kMaxExperts];
+    __shared__ int sCount[kMaxExperts];
+    __shared__ double sP[kMaxExperts];
+    const int e = threadIdx.x;
+    if (e < a.E) {
+        int base = 0, total = 0;
+        double ps = 0.0;
+        for (int r = 0; r < a.world; ++r) {
+            const int c = a.all_counts[(int64_t)r * a.E + e];
+            if (r < a.rank) base += c;
+            total += c;
+            ps += a.all_psum[(int64_t)r * a.E + e];
+        }
+        const int mine = a.all_counts[(int64_t)a.rank * a.E + e];
+        const int left = a.cap - base > 0 ? a.cap - base : 0;
+        a.cap_e[e] = left;
+        sKept[e] = mine < left ? mine : left;
+        sCount[e] = total;
+        sP[e] = a.T_global > 0 ? ps / (double)a.T_global : 0.0;
+    }
+    __syncthreads();
+    if (e == 0) {
+        int off = 0;
+        double l = 0.0;
+        for (int i = 0; i < a.E; ++i) {
+            a.offsets[i] = off;
+            off += sKept[i];
+            a.counts[i] = sCount[i];
+            const double f = a.T_global > 0 ? (double)sCount[i] / ((double)a.T_global * a.k) : 0.0;
+            a.f[i] = (float)f;
+            a.p[i] = (float)sP[i];
+            l += f * sP[i];
+        }
+        a.offsets[a.E] = off;
+        a.l_aux[0] = (float)((double)a.alpha * a.E * l);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s) {
+    dp_prepare_kernel<<<1, 64, 0, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s) {
     const int nchunk = (int)((T + kChunkTokens - 1) / kChunkTokens);

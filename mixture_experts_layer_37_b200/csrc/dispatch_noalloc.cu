@@ -90,6 +90,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     sa.f = nullptr;
     sa.p = nullptr;
     sa.l_aux = nullptr;
+    sa.psum_total = nullptr;
     sa.T = cfg->T;
     sa.nchunk = (int)nchunk;
     sa.E = cfg->E;
@@ -105,6 +106,7 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     xa.src_assign = src_assign;
     xa.x = x;
     xa.x_perm = x_perm;
+    xa.cap_e = nullptr;
     xa.T = cfg->T;
     xa.E = cfg->E;
     xa.k = cfg->k;

@@ -10,6 +10,9 @@
 // (discosf.com/news/5228035) §2.1), and all tokens of one expert processed as
 // one matrix product (MoE-basics §4.4).
 //
+// This file: the one-CTA-per-tile kernel and the host launcher; the CTA-pair
+// kernel (cta_group::2, 256-row tiles) is in gemm_sm100_pair.cu.
+//
 // Kernel design (one persistent CTA per SM, 192 threads):
 //   warp 0   TMA producer: A tile [128 rows x 64 K] of the expert-sorted
 //            activations (K-major, 128-byte swizzle) and four [64 K x 64 N]
@@ -29,56 +32,20 @@
 // reads the next rows (or TMA zero-fill) and masks them at the store.
 // Every wait is bounded in time; on expiry the kernel records a timeout,
 // drains its own copies and MMAs, frees TMEM and returns.
-#include "internal.h"
+#include "gemm_common.cuh"
 
 namespace moe {
 namespace {
 
+using namespace gemm;
+
 constexpr int BM = 128;
-constexpr int BK = 64;
-constexpr int BN_MMA = 256;
 constexpr int kStages = 4;
 constexpr int kAStageBytes = BM * BK * 2;                  // 16 KB
-constexpr int kBBoxBytes = BK * 64 * 2;                    // 8 KB: 64 K-rows x 64 N (128 B)
 constexpr int kBStageBytes = 4 * kBBoxBytes;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;   // 48 KB
-constexpr int kTmemCols = 2 * BN_MMA;                      // two fp32 accumulators
-constexpr int kThreads = 192;
-constexpr int kGroupM = 32;  // m-tiles per raster group
-constexpr int kBiasBytes = 4 * BN_MMA * 2;                 // one bf16 bias row per epilogue warp
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + 1024 /*alignment*/;
-
-enum { MODE_PLAIN = 0, MODE_SWIGLU = 1, MODE_GELU = 2 };
-
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
-// = 1), B bf16 (bits 10-12 = 1), A K-major (bit 15 = 0), B MN-major (bit 16
-// = 1), N>>3 in bits 17-22, M>>4 in bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            ((uint32_t)(BN_MMA >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-
-// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading
-// and stride byte offsets (all >> 4), version 1 (bit 46), layout 2 (bits 61-63).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
-    return d;
-}
-
-struct GemmParams {
-    const int32_t* offsets;      // [E+1] kept-row offsets per expert
-    __nv_bfloat16* out;          // [rows_cap, N]
-    const __nv_bfloat16* bias;   // [E, N] or null
-    int E, K, N;
-    int bn_out;                  // output columns per tile: 128 (SwiGLU) or 256
-    int n_tiles;
-    DevStatus st;
-};
-
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
-__device__ __forceinline__ float gelu_f(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+constexpr uint32_t kIdesc = make_idesc(BM, BN_MMA);
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -123,17 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (threadIdx.x == 64) {
-        int acc = 0;
-        mt_prefix[0] = 0;
-        for (int e = 0; e < p.E; ++e) {
-            const int o0 = p.offsets[e], o1 = p.offsets[e + 1];
-            s_off[e] = o0;
-            acc += (o1 - o0 + BM - 1) / BM;
-            mt_prefix[e + 1] = acc;
-        }
-        s_off[p.E] = p.offsets[p.E];
-    }
+    if (threadIdx.x == 64) build_tile_table(p, BM, mt_prefix, s_off);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -142,24 +99,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kblocks = p.K / BK;
     const uint64_t tmo = p.st.timeout_ns;
 
-    // Tile order: expert by expert; inside an expert, groups of kGroupM
-    // m-tiles, and inside a group n-tile-major.  The CTAs running at the same
-    // time then share each weight tile among up to kGroupM of them and each
-    // activation tile among the group's n-tiles, which keeps the expert's
-    // working set in L2 even when its weights exceed it.
-    auto decode = [&](int tile, int& e, int& row0, int& rows, int& nt) {
-        e = 0;
-        while (mt_prefix[e + 1] * p.n_tiles <= tile) ++e;
-        const int local = tile - mt_prefix[e] * p.n_tiles;
-        const int mt_e = mt_prefix[e + 1] - mt_prefix[e];
-        const int grp = local / (kGroupM * p.n_tiles);
-        const int gm = min(kGroupM, mt_e - grp * kGroupM);
-        const int r = local - grp * kGroupM * p.n_tiles;
-        nt = r / gm;
-        const int mt = grp * kGroupM + (r - nt * gm);
-        row0 = s_off[e] + mt * BM;
-        rows = min(BM, s_off[e + 1] - row0);
-    };
     auto give_up = [&](uint32_t site) {
         report_timeout(p.st, site);
         *abort_flag = 1;
@@ -174,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool stop = false;
             for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
                 int e, row0, rows, nt;
-                decode(tile, e, row0, rows, nt);
+                decode_tile(tile, mt_prefix, s_off, p.n_tiles, BM, e, row0, rows, nt);
                 const int n0 = nt * p.bn_out;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (*abort_flag) { stop = true; break; }
@@ -263,13 +202,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
+        __nv_bfloat16* wb = s_bias + (warp - 2) * BN_MMA;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
             const int ab = __shfl_sync(0xffffffffu, *abort_flag, 0);
             if (ab) break;
             int e, row0, rows, nt;
-            decode(tile, e, row0, rows, nt);
+            decode_tile(tile, mt_prefix, s_off, p.n_tiles, BM, e, row0, rows, nt);
             const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, tmo);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) give_up(SITE_GEMM_EPI_TMEM_FULL);
@@ -280,63 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = r < rows;
             __nv_bfloat16* orow = p.out + (int64_t)(row0 + (valid ? r : 0)) * p.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
-            const int n0 = nt * p.bn_out;
-            if (MODE == MODE_SWIGLU) {
-                for (int c = 0; c < 128; c += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld_16(tbase + c, g);
-                    tmem_ld_16(tbase + 128 + c, u);
-                    tmem_ld_wait();
-                    if (valid && n0 + c < p.N) {
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                            const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-                            pk[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + n0 + c);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
-                }
-            } else {
-                // this tile's 256 bias values, staged once per tile in the warp's own row
-                __nv_bfloat16* wb = s_bias + (warp - 2) * BN_MMA;
-                if (p.bias != nullptr) {
-                    __syncwarp();
-                    const int col = n0 + 8 * lane;
-                    uint4 bv = make_uint4(0, 0, 0, 0);
-                    if (col < p.N) bv = *reinterpret_cast<const uint4*>(p.bias + (int64_t)e * p.N + col);
-                    reinterpret_cast<uint4*>(wb)[lane] = bv;
-                    __syncwarp();
-                }
-                for (int c = 0; c < BN_MMA; c += 16) {
-                    uint32_t v[16];
-                    tmem_ld_16(tbase + c, v);
-                    tmem_ld_wait();
-                    if (valid && n0 + c < p.N) {
-                        float x[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(v[i]);
-                        if (p.bias != nullptr) {
-                            const __nv_bfloat16* b = wb + c;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] += __bfloat162float(b[i]);
-                        }
-                        if (MODE == MODE_GELU) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] = gelu_f(x[i]);
-                        }
-                        uint32_t pk[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-                        uint4* dst = reinterpret_cast<uint4*>(orow + n0 + c);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
-                }
-            }
+            epilogue_rows<MODE>(p, tbase, orow, valid, nt * p.bn_out, e, wb, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -369,8 +253,28 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous, row pitch `pitch` bytes),
-// box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+template <int MODE>
+cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
+                        int64_t rows_cap, cudaStream_t s) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 64 || !attr_set[dev]) {
+        cudaError_t err =
+            cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (err != cudaSuccess) return err;
+        if (dev < 64) attr_set[dev] = true;
+    }
+    const int64_t tiles_upper = (rows_cap / BM + p.E) * (int64_t)p.n_tiles;
+    const int grid = (int)min64(tiles_upper, (int64_t)sm_count());
+    if (grid <= 0) return cudaSuccess;
+    grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+namespace gemm {
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch, uint32_t box_inner,
               uint32_t box_outer) {
     EncodeTiledFn enc = encode_fn();
@@ -383,39 +287,51 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+}  // namespace gemm
 
-template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
-                        int64_t rows_cap, cudaStream_t s) {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t err =
-            cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        attr_set[dev] = true;
+// CTA-pair variant (gemm_sm100_pair.cu).
+cudaError_t launch_pair_gemm(int mode, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                             const gemm::GemmParams& p, int64_t rows_cap, cudaStream_t s);
+
+namespace {
+// Kernel choice per GEMM.  The CTA pair halves the weight bytes each SM loads
+// and reads per MMA, but pads each expert's rows to 256 instead of 128.  It is
+// used for the second GEMM and for the GELU first GEMM (long K per tile or a
+// heavy epilogue), and when an expert is expected to hold at least 512 rows;
+// the one-CTA kernel for the SwiGLU first GEMM and for small batches.
+// MOE_GEMM_CTA_PAIR=0/1 forces one kernel (benchmarking).
+int forced_variant() {
+    static int v = -2;
+    if (v == -2) {
+        const char* env = getenv("MOE_GEMM_CTA_PAIR");
+        v = env == nullptr ? -1 : (env[0] == '0' ? 0 : 1);
     }
-    const int64_t tiles_upper = (rows_cap / BM + p.E) * (int64_t)p.n_tiles;
-    const int grid = (int)min64(tiles_upper, (int64_t)sm_count());
-    if (grid <= 0) return cudaSuccess;
-    grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
-    return cudaGetLastError();
+    return v;
 }
 
+cudaError_t launch_one(int mode, bool pair_ok, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const GemmParams& p, int64_t rows_cap, cudaStream_t s) {
+    const int f = forced_variant();
+    const bool pair = f >= 0 ? f == 1 : (pair_ok && mode != MODE_SWIGLU);
+    if (pair) return launch_pair_gemm(mode, a, b0, b1, p, rows_cap, s);
+    if (mode == MODE_SWIGLU) return launch_mode<MODE_SWIGLU>(a, b0, b1, p, rows_cap, s);
+    if (mode == MODE_GELU) return launch_mode<MODE_GELU>(a, b0, b1, p, rows_cap, s);
+    return launch_mode<MODE_PLAIN>(a, b0, b1, p, rows_cap, s);
+}
 }  // namespace
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     if (a.rows_cap <= 0) return cudaSuccess;
     const bool swiglu = a.act == 0;
+    // A maps use 128-row boxes (one CTA's half of a pair tile, or a whole single-CTA tile)
     CUtensorMap mA1, mB1, mB1u, mA2, mB2;
-    bool ok = make_map(&mA1, a.x_perm, (uint64_t)a.d, (uint64_t)a.rows_cap, (uint64_t)a.d * 2, 64, BM);
+    bool ok = make_map(&mA1, a.x_perm, (uint64_t)a.d, (uint64_t)a.rows_cap, (uint64_t)a.d * 2, 64, 128);
     ok = ok && make_map(&mB1, a.w1, (uint64_t)a.ffn, (uint64_t)a.E * a.d, (uint64_t)a.ffn * 2, 64, BK);
     if (swiglu)
         ok = ok && make_map(&mB1u, a.w_up, (uint64_t)a.ffn, (uint64_t)a.E * a.d, (uint64_t)a.ffn * 2, 64, BK);
     else
         mB1u = mB1;
-    ok = ok && make_map(&mA2, a.h, (uint64_t)a.ffn, (uint64_t)a.rows_cap, (uint64_t)a.ffn * 2, 64, BM);
+    ok = ok && make_map(&mA2, a.h, (uint64_t)a.ffn, (uint64_t)a.rows_cap, (uint64_t)a.ffn * 2, 64, 128);
     ok = ok && make_map(&mB2, a.w2, (uint64_t)a.d, (uint64_t)a.E * a.ffn, (uint64_t)a.d * 2, 64, BK);
     if (!ok) return cudaErrorInvalidValue;
 
@@ -429,8 +345,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p1.bn_out = swiglu ? 128 : 256;
     p1.n_tiles = (a.ffn + p1.bn_out - 1) / p1.bn_out;
     p1.st = a.st;
-    cudaError_t err = swiglu ? launch_mode<MODE_SWIGLU>(mA1, mB1, mB1u, p1, a.rows_cap, s)
-                             : launch_mode<MODE_GELU>(mA1, mB1, mB1u, p1, a.rows_cap, s);
+    // rows an expert is expected to receive (the routing itself stays on the device)
+    const bool pair_ok = a.rows_cap / a.E >= 512;
+    cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair_ok, mA1, mB1, mB1u, p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
     if (a.between != nullptr && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
 
@@ -444,7 +361,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p2.bn_out = 256;
     p2.n_tiles = (a.d + 255) / 256;
     p2.st = a.st;
-    return launch_mode<MODE_PLAIN>(mA2, mB2, mB2, p2, a.rows_cap, s);
+    return launch_one(MODE_PLAIN, pair_ok, mA2, mB2, mB2, p2, a.rows_cap, s);
 }
 
 }  // namespace moe

@@ -19,6 +19,7 @@ struct ScanArgs {
     float* f;              // [E] out or null
     float* p;              // [E] out or null
     float* l_aux;          // [1] out or null
+    double* psum_total;    // [E] out or null: sum over this batch's tokens of p[t,e] (not divided)
     int64_t T;
     int nchunk, E, k, cap;
     float alpha;
@@ -57,11 +58,30 @@ struct ScatterArgs {
     int32_t* src_assign;        // [R_max]
     const void* x;              // [T, d]
     void* x_perm;               // [R_max, d]
+    const int32_t* cap_e;       // [E] per-expert capacity left for this batch, or null (use cap)
     int64_t T;
     int E, k, cap, nchunk;
     int row_bytes;              // d * element size (multiple of 16)
 };
 cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
+
+// Data-parallel shard of one logical batch: from every rank's counts and
+// probability sums ([world, E], gathered in rank order) compute this rank's
+// per-expert capacity left, kept offsets, and the global counts / f / p / L_aux.
+struct DpPrepareArgs {
+    const int32_t* all_counts;  // [world, E]
+    const double* all_psum;     // [world, E]
+    int world, rank, E, k, cap;
+    int64_t T_global;
+    float alpha;
+    int32_t* cap_e;             // [E] out
+    int32_t* offsets;           // [E+1] out (this rank's kept rows)
+    int32_t* counts;            // [E] out (global)
+    float* f;                   // [E] out
+    float* p;                   // [E] out
+    float* l_aux;               // [1] out
+};
+cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s);
 
 struct CombineArgs {
     const void* y_perm;    // [R_max, d]

@@ -80,13 +80,13 @@ int64_t max_rows(const moe_config_t* c) {
 struct Plan {
     int nchunk;
     int64_t rows;
-    size_t hist, psum, base, xperm, h, yperm, total;
+    size_t hist, psum, base, cap_e, xperm, h, yperm, total;
 };
 
-Plan plan_of(const moe_config_t* c) {
+Plan plan_rows(const moe_config_t* c, int64_t rows) {
     Plan p;
     p.nchunk = (int)((c->T + kChunkTokens - 1) / kChunkTokens);
-    p.rows = max_rows(c);
+    p.rows = rows;
     const size_t s = elem_size(c);
     const size_t E = (size_t)c->E;
     size_t off = kStatusBytes;
@@ -96,6 +96,8 @@ Plan plan_of(const moe_config_t* c) {
     off = align_up(off + (size_t)p.nchunk * E * 8, 1024);
     p.base = off;
     off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
+    p.cap_e = off;
+    off = align_up(off + E * 4, 1024);
     p.xperm = off;
     off = align_up(off + (size_t)p.rows * c->d * s, 1024);
     p.h = off;
@@ -104,6 +106,34 @@ Plan plan_of(const moe_config_t* c) {
     off = align_up(off + (size_t)p.rows * c->d * s, 1024);
     p.total = off;
     return p;
+}
+
+Plan plan_of(const moe_config_t* c) { return plan_rows(c, max_rows(c)); }
+
+// Data-parallel shard of a batch of T_global tokens: capacity of the whole
+// batch, and the most rows this shard can keep.
+int64_t dp_cap_used(const moe_config_t* c, int64_t T_global) {
+    moe_config_t g = *c;
+    g.T = T_global;
+    const int64_t cap = capacity_formula(&g);
+    return cap < T_global ? cap : T_global;
+}
+int64_t dp_rows(const moe_config_t* c, int64_t T_global) {
+    int64_t cap = dp_cap_used(c, T_global);
+    if (cap > c->T) cap = c->T;
+    const int64_t a = c->T * c->k, b = (int64_t)c->E * cap;
+    return a < b ? a : b;
+}
+moe_status_t check_dp(const moe_config_t* c, int64_t T_global) {
+    if (T_global < c->T) return MOE_ERR_INVALID_ARG;
+    if (T_global * (int64_t)c->k >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status_t check_ws_plan(const Plan& pl, const void* ws, size_t ws_bytes) {
+    if (ws == nullptr || ws_bytes < pl.total) return MOE_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 1023u) != 0) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
 }
 
 moe_status_t check_ws(const moe_config_t* c, const void* ws, size_t ws_bytes, Plan* p) {
@@ -151,6 +181,7 @@ ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, flo
     sa.f = f;
     sa.p = p;
     sa.l_aux = l_aux;
+    sa.psum_total = nullptr;
     sa.T = c->T;
     sa.nchunk = pl.nchunk;
     sa.E = c->E;
@@ -187,7 +218,8 @@ moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_rout
 }
 
 moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* idx, const int32_t* offsets,
-                         int32_t* slot, int32_t* src_assign, void* x_perm, void* ws, const Plan& pl, cudaStream_t s) {
+                         int32_t* slot, int32_t* src_assign, void* x_perm, void* ws, const Plan& pl, cudaStream_t s,
+                         const int32_t* cap_e = nullptr) {
     ScatterArgs xa;
     xa.topk_idx = idx;
     xa.chunk_base = reinterpret_cast<const int32_t*>(at(ws, pl.base));
@@ -196,6 +228,7 @@ moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* id
     xa.src_assign = src_assign;
     xa.x = x;
     xa.x_perm = x_perm;
+    xa.cap_e = cap_e;
     xa.T = c->T;
     xa.E = c->E;
     xa.k = c->k;
@@ -404,6 +437,90 @@ moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* 
                                   cudaStream_t stream, cudaEvent_t* stage_events) {
     if (stage_events == nullptr) return MOE_ERR_INVALID_ARG;
     return forward_impl(cfg, weights, x, logits_in, o, ws, ws_bytes, stream, stage_events);
+}
+
+moe_status_t moe_dp_workspace_size(const moe_config_t* cfg, int64_t T_global, size_t* bytes) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+    *bytes = plan_rows(cfg, dp_rows(cfg, T_global)).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_dp_max_rows(const moe_config_t* cfg, int64_t T_global, int64_t* rows) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
+    if (rows == nullptr) return MOE_ERR_INVALID_ARG;
+    *rows = dp_rows(cfg, T_global);
+    return MOE_OK;
+}
+
+moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_weights_t* weights, const void* x,
+                          const float* logits_in, moe_outputs_t* o, int32_t* local_counts, double* local_psum,
+                          void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
+    if ((st = check_weights(cfg, weights, logits_in == nullptr, false)) != MOE_OK) return st;
+    if (o == nullptr || o->offsets == nullptr || local_counts == nullptr || local_psum == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->topk_idx == nullptr || o->topk_w == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const Plan pl = plan_rows(cfg, dp_rows(cfg, T_global));
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    ScanArgs sa = scan_args(cfg, local_counts, o->offsets, nullptr, nullptr, nullptr, true, ws, pl);
+    sa.cap = 0x7fffffff;        // local totals only; the capacity is applied in moe_dp_finish
+    sa.psum_total = local_psum;
+    if (cfg->T == 0) return from_cuda(launch_dispatch_scan(sa, stream));
+    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
+                      o->logits_out, o->probs_out, ws, pl, stream, &sa);
+}
+
+moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
+                           const double* all_psum, int32_t world, int32_t rank, const moe_weights_t* weights,
+                           const void* x, moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
+    if ((st = check_weights(cfg, weights, false, true)) != MOE_OK) return st;
+    if (world < 1 || rank < 0 || rank >= world || all_counts == nullptr || all_psum == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (o == nullptr || o->counts == nullptr || o->offsets == nullptr || o->f == nullptr || o->p == nullptr ||
+        o->l_aux == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->out == nullptr || !aligned16(o->out) ||
+                       o->topk_idx == nullptr || o->topk_w == nullptr || o->slot == nullptr ||
+                       o->src_assign == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const Plan pl = plan_rows(cfg, dp_rows(cfg, T_global));
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    DpPrepareArgs dp;
+    dp.all_counts = all_counts;
+    dp.all_psum = all_psum;
+    dp.world = world;
+    dp.rank = rank;
+    dp.E = cfg->E;
+    dp.k = cfg->k;
+    dp.cap = (int)dp_cap_used(cfg, T_global);
+    dp.T_global = T_global;
+    dp.alpha = cfg->aux_alpha;
+    dp.cap_e = reinterpret_cast<int32_t*>(at(ws, pl.cap_e));
+    dp.offsets = o->offsets;
+    dp.counts = o->counts;
+    dp.f = o->f;
+    dp.p = o->p;
+    dp.l_aux = o->l_aux;
+    if (launch_dp_prepare(dp, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cfg->T == 0) return MOE_OK;
+    void* x_perm = at(ws, pl.xperm);
+    void* y_perm = at(ws, pl.yperm);
+    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, x_perm, ws, pl, stream, dp.cap_e);
+    if (st != MOE_OK) return st;
+    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream);
+    if (st != MOE_OK) return st;
+    return run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
 }
 
 moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_host,

@@ -9,10 +9,11 @@
 // "Llama-MoE架构解析" (coreui.cn/article/2610641) §3.1 (softmax -> top-k ->
 // divide by the sum of the k weights).
 //
-// bf16: one CTA of 8 warps per `tpc` tokens (32, 64 or 128: enough CTAs to
+// bf16: one CTA of 8 warps per `tpc` tokens (32 or 64: enough CTAs to
 // fill the GPU, and enough tokens per CTA that re-reading the router weight
 // per CTA stays small next to the x stream).  The warps form tpc/16 token
-// groups x 128/tpc K-splits.  Each warp streams its x rows once from HBM with
+// groups x 128/tpc K-splits; each token's logits are always the same
+// fixed-order sum of four K partial sums, so they do not depend on the batch.  Each warp streams its x rows once from HBM with
 // 16-byte loads, four 32-column blocks (8 loads per lane) in flight per batch
 // and two CTAs per SM, and multiplies on the tensor cores with mma.sync m16n8k16 (bf16 in,
 // fp32 accumulate).  The router weight [d, E] is copied into shared memory as
@@ -34,7 +35,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kLStride = kMaxExperts + 1;
 constexpr int kSlabBytes = 64 * 1024;
-constexpr int kMaxTpc = 128;
+constexpr int kMaxTpc = 64;
+constexpr int kSplits = 4;  // K partial sums per token, always (batch-invariant logits)
 constexpr int kBatch = 4;  // 32-column blocks of x loaded per batch
 
 __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
@@ -169,7 +171,7 @@ struct SlabGeom {
     static constexpr int kUnits = (NT & 1) ? NT : NT + 1;   // odd row pitch in 16-byte units
     static constexpr int kPitch = 16 * kUnits;
     static constexpr int kRows = (kSlabBytes / kPitch) / 128 * 128;
-    static constexpr int kPartBytes = 128 * 8 * NT * 4;     // nsplit * tpc = 128 rows of EP floats
+    static constexpr int kPartBytes = kSplits * kMaxTpc * 8 * NT * 4;  // [4][tpc][EP] floats
 };
 
 // Bytes of the shared region that holds the weight slab, and after the K
@@ -185,7 +187,7 @@ __host__ __device__ __forceinline__ int tail_bytes_for(int tpc) {
     return tpc * kLStride * 4 + (kMaxTpc / kChunkTokens) * kMaxExperts * 4;
 }
 
-template <int NT>  // experts padded to 8*NT
+template <int NT, int TPC>  // experts padded to 8*NT; TPC tokens per CTA (32 or 64)
 __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) {
     using G = SlabGeom<NT>;
     constexpr int EP = 8 * NT;
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int ngroups = a.tpc / 16, nsplit = 8 / ngroups;
+    constexpr int ngroups = TPC / 16, nsplit = 8 / ngroups, kSets = kSplits / nsplit;
     const int tg = warp % ngroups, ksplit = warp / ngroups;
     const int E = a.E, d = a.d;
     const int64_t t0 = (int64_t)blockIdx.x * a.tpc;
@@ -218,9 +220,15 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
     const int la = lr >> 1, lb = 2 * lj + (lr & 1);
     const uint32_t lds_base = smem_u32(sW) + (uint32_t)((8 * la + ((lb + 2 * la) & 7)) * G::kPitch);
 
-    float acc[NT][4];
+    // Every token's logits are the fixed-order sum of kSplits partial sums,
+    // partial s accumulating the 32-column blocks b with b % 4 == s in
+    // ascending order; a warp owns partials ksplit + nsplit*j.  The result is
+    // therefore independent of how tokens are grouped into CTAs (batch size).
+    float acc[kSets][NT][4];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int j = 0; j < kSets; ++j)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) acc[j][n][0] = acc[j][n][1] = acc[j][n][2] = acc[j][n][3] = 0.f;
 
     const bool vec_rows = (E & 7) == 0;
     for (int k0 = 0; k0 < d; k0 += G::kRows) {
@@ -271,35 +279,40 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
             for (int u = 0; u < kBatch; ++u) {
                 const int blk = b0 + u * nsplit;
                 if (blk >= nblk) break;
+                // which of this warp's partials: (blk % 4) = ksplit + nsplit * j.  With
+                // kBatch a multiple of kSets, j is fixed by u at compile time.
+                const int j = ((u * nsplit) % kSplits) / nsplit;
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     uint32_t b0r, b1r, b2r, b3r;
                     ldsm_x4_trans(lds_base + (uint32_t)(32 * blk * G::kPitch + 16 * n), b0r, b1r, b2r, b3r);
-                    mma_bf16_16816(acc[n], xa[u].x, xb[u].x, xa[u].y, xb[u].y, b0r, b1r);
-                    mma_bf16_16816(acc[n], xa[u].z, xb[u].z, xa[u].w, xb[u].w, b2r, b3r);
+                    mma_bf16_16816(acc[j][n], xa[u].x, xb[u].x, xa[u].y, xb[u].y, b0r, b1r);
+                    mma_bf16_16816(acc[j][n], xa[u].z, xb[u].z, xa[u].w, xb[u].w, b2r, b3r);
                 }
             }
         }
     }
     __syncthreads();  // the slab region is reused for the partials
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const int e0 = n * 8 + 2 * c;
-        float* pa = sPart + (ksplit * a.tpc + tg * 16 + g) * EP;
-        float* pb = pa + 8 * EP;
-        pa[e0] = acc[n][0];
-        pa[e0 + 1] = acc[n][1];
-        pb[e0] = acc[n][2];
-        pb[e0 + 1] = acc[n][3];
+    for (int j = 0; j < kSets; ++j) {
+        const int sidx = ksplit + nsplit * j;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int e0 = n * 8 + 2 * c;
+            float* pa = sPart + (sidx * a.tpc + tg * 16 + g) * EP;
+            float* pb = pa + 8 * EP;
+            pa[e0] = acc[j][n][0];
+            pa[e0 + 1] = acc[j][n][1];
+            pb[e0] = acc[j][n][2];
+            pb[e0 + 1] = acc[j][n][3];
+        }
     }
     __syncthreads();
     const int split_stride = a.tpc * EP;
     for (int i = tid; i < a.tpc * E; i += kThreads) {
         const int tok = i / E, e = i - tok * E;
         const float* p = sPart + tok * EP + e;
-        float v = p[0];
-        for (int s = 1; s < nsplit; ++s) v += p[s * split_stride];
-        sL[tok * kLStride + e] = v;
+        sL[tok * kLStride + e] = ((p[0] + p[split_stride]) + p[2 * split_stride]) + p[3 * split_stride];
     }
     __syncthreads();
     router_finish(a, sL, sHist, true);
@@ -352,33 +365,39 @@ __global__ void __launch_bounds__(kThreads) router_f32_kernel(RouterArgs a) {
     router_finish(a, sL, sHist, true);
 }
 
-// Tokens per CTA: at least 4E (router weight re-read per CTA <= 1/4 of its
-// x bytes), at most 128, and small enough to give >= ~1 CTA per SM.
+// Tokens per CTA: 64 when 16 < E <= 32 (router weight re-read per CTA at most
+// half of its x bytes) and there are enough tokens for >= ~1 CTA per SM,
+// else 32.
 int pick_tpc(int64_t T, int E) {
-    int tpc = 32;
-    while (tpc < 4 * E && tpc < kMaxTpc) tpc *= 2;
-    const int64_t sms = sm_count();
-    while (tpc > 32 && (T + tpc - 1) / tpc < sms) tpc /= 2;
-    return tpc;
+    if (E > 16 && E <= 32 && (T + 63) / 64 >= sm_count()) return 64;
+    return 32;
 }
 
-template <int NT>
-cudaError_t launch_bf16_nt(RouterArgs a, cudaStream_t s) {
-    a.tpc = pick_tpc(a.T, a.E);
-    const size_t smem = (size_t)union_bytes_for<NT>(a.d) + tail_bytes_for(a.tpc);
+template <int NT, int TPC>
+cudaError_t launch_bf16_tpc(RouterArgs a, cudaStream_t s) {
+    a.tpc = TPC;
+    const size_t smem = (size_t)union_bytes_for<NT>(a.d) + tail_bytes_for(TPC);
     const size_t smem_max = (size_t)union_bytes_for<NT>(1 << 30) + tail_bytes_for(kMaxTpc);
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr[dev]) {
-        cudaError_t err =
-            cudaFuncSetAttribute(router_bf16_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+        cudaError_t err = cudaFuncSetAttribute(router_bf16_kernel<NT, TPC>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
         if (err != cudaSuccess) return err;
         if (dev < 64) attr[dev] = true;
     }
-    const int grid = (int)((a.T + a.tpc - 1) / a.tpc);
-    router_bf16_kernel<NT><<<grid, kThreads, smem, s>>>(a);
+    const int grid = (int)((a.T + TPC - 1) / TPC);
+    router_bf16_kernel<NT, TPC><<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int NT>
+cudaError_t launch_bf16_nt(RouterArgs a, cudaStream_t s) {
+    if constexpr (NT == 3 || NT == 4) {
+        if (pick_tpc(a.T, a.E) == 64) return launch_bf16_tpc<NT, 64>(a, s);
+    }
+    return launch_bf16_tpc<NT, 32>(a, s);
 }
 
 template <int EP>

@@ -71,6 +71,7 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
         if (lane == 0) {
             sCount[e] = run;
             sP[e] = (pp != nullptr && a.T > 0) ? ps / (double)a.T : 0.0;
+            if (a.psum_total != nullptr) a.psum_total[e] = ps;
         }
     }
     __syncthreads();

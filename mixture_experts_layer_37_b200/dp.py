@@ -1,0 +1,74 @@
+"""Data-parallel sharding of one logical MoE batch over torch.distributed ranks.
+
+Each rank holds a contiguous slice of the batch (slices in rank order).  The
+capacity cut and the load-balance statistics are those of the whole batch: the
+per-expert counts and probability sums of every slice are all-gathered (the
+exchange that data-parallel MoE training does before its load-balance loss,
+"Hand-building a LLaMA4-MoE" (dpshk.com/news/5809432) §3.1), and the second
+phase on each rank keeps only the capacity left after the lower ranks'
+assignments.  The collectives are two all-gathers of E numbers per rank (NCCL
+over NVLink on GPUs); the computation before and after runs in libmoe's
+kernels (moe_dp_route, moe_dp_finish).
+"""
+from __future__ import annotations
+
+from typing import Callable, Optional
+
+import torch
+import torch.distributed as dist
+
+from . import (MoEConfig, Workspace, allocate_outputs, moe_dp_finish, moe_dp_max_rows, moe_dp_route,
+               moe_dp_workspace_size)
+
+
+def gather_rank_order(t: torch.Tensor, world: int, group=None) -> torch.Tensor:
+    """[world, *t.shape] with rank r's tensor in row r."""
+    parts = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(parts, t.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+class DataParallelMoE:
+    """One rank's share of a data-parallel MoE layer forward.
+
+    `route` and `finish` default to the library's two phases; tests of the
+    orchestration on CPU ranks may substitute stand-ins with the same
+    signatures."""
+
+    def __init__(self, cfg_local: MoEConfig, weights: dict, group=None, device="cuda",
+                 route: Optional[Callable] = None, finish: Optional[Callable] = None, T_global: Optional[int] = None):
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.cfg = cfg_local
+        self.weights = weights
+        if T_global is None:
+            t = torch.tensor([cfg_local.T], dtype=torch.int64, device=device)
+            dist.all_reduce(t, group=self.group)
+            T_global = int(t.item())
+        self.T_global = T_global
+        self._route = route or self._lib_route
+        self._finish = finish or self._lib_finish
+        self.device = device
+        if route is None or finish is None:
+            self.outputs = allocate_outputs(cfg_local, device)
+            rows = max(moe_dp_max_rows(cfg_local, T_global), 1)
+            self.outputs["src_assign"] = torch.empty(rows, dtype=torch.int32, device=device)
+            self.ws = Workspace(cfg_local, device, nbytes=moe_dp_workspace_size(cfg_local, T_global))
+        self.local_counts = torch.zeros(cfg_local.E, dtype=torch.int32, device=device)
+        self.local_psum = torch.zeros(cfg_local.E, dtype=torch.float64, device=device)
+
+    def _lib_route(self, x, logits_in):
+        moe_dp_route(self.cfg, self.T_global, self.weights, x, self.outputs, self.local_counts, self.local_psum,
+                     self.ws, logits_in)
+
+    def _lib_finish(self, x, all_counts, all_psum):
+        moe_dp_finish(self.cfg, self.T_global, all_counts, all_psum, self.world, self.rank, self.weights, x,
+                      self.outputs, self.ws)
+        return self.outputs
+
+    def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None) -> dict:
+        self._route(x_local, logits_in)
+        all_counts = gather_rank_order(self.local_counts, self.world, self.group)
+        all_psum = gather_rank_order(self.local_psum, self.world, self.group)
+        return self._finish(x_local, all_counts, all_psum)

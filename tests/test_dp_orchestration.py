@@ -1,0 +1,109 @@
+"""Data-parallel sharding of one batch, on CPU ranks (gloo, world sizes 2 and 3).
+
+The orchestration of mixture_experts_layer_37_b200.dp (slice order, the two
+all-gathers in rank order, the whole-batch token count) runs for real over
+torch.distributed; the two device phases are replaced by stand-ins built from
+the oracle, so no GPU is needed.  The stand-in finish phase applies the rule
+the device phase implements: rank r may keep max(0, cap - base_e) rows of
+expert e, base_e = assignments to e on lower ranks.  The test checks that the
+sharded result equals the oracle's dispatch and statistics of the whole batch."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, bounds, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import workloads as W
+    from oracle import moe_oracle as O
+    from mixture_experts_layer_37_b200 import MoEConfig
+    from mixture_experts_layer_37_b200.dp import DataParallelMoE
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = W.Workload("dp", T=bounds[-1], d=32, ffn=64, E=6, k=2, act="swiglu", dtype="f32",
+                        capacity_factor=0.7, zipf_router_bias=True, seed=31, w_std=0.2)
+        inp = W.make_inputs(wl, with_experts=False)
+        t0, t1 = bounds[rank], bounds[rank + 1]
+        full = O.route(wl, inp)
+        logits_local = full["logits"][t0:t1]
+        cap = O.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+        state = {}
+
+        def route(x, logits_in):
+            p = O.softmax(logits_local)
+            idx = O.select_topk(logits_local, wl.k)
+            state["idx"] = idx
+            dp.local_counts.copy_(torch.from_numpy(np.bincount(idx.reshape(-1), minlength=wl.E).astype(np.int32)))
+            dp.local_psum.copy_(torch.from_numpy(p.sum(axis=0)))
+
+        def finish(x, all_counts, all_psum):
+            ac = all_counts.numpy().astype(np.int64)
+            base = ac[:rank].sum(axis=0)
+            cap_left = np.maximum(0, cap - base)
+            d = O.dispatch(state["idx"], wl.E, 10 ** 9)
+            kept = d["rank"] < cap_left[state["idx"]]
+            gcounts = ac.sum(axis=0)
+            f, pm, l = O.aux_stats(gcounts, np.zeros((0, wl.E)), wl.T, wl.k, wl.aux_alpha)
+            pm = all_psum.numpy().sum(axis=0) / wl.T
+            l = wl.aux_alpha * wl.E * float(np.sum(f * pm))
+            return {"kept": kept, "counts": gcounts, "f": f, "p": pm, "l_aux": l}
+
+        cfg = MoEConfig(T=t1 - t0, d=wl.d, ffn=wl.ffn, E=wl.E, k=wl.k, dtype="f32", capacity_factor=wl.capacity_factor)
+        dp = DataParallelMoE(cfg, {}, device="cpu", route=route, finish=finish)
+        assert dp.T_global == wl.T and dp.world == world and dp.rank == rank
+        res = dp.forward(torch.zeros((t1 - t0, wl.d)))
+        q.put((rank, res["kept"], res["counts"], res["f"], res["p"], res["l_aux"]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("bounds", [[0, 120, 257], [0, 50, 51, 200]], ids=["world2", "world3"])
+def test_sharded_batch_equals_whole_batch(bounds):
+    import workloads as W
+    from oracle import moe_oracle as O
+
+    world = len(bounds) - 1
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, bounds, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    for _ in range(world):
+        r, kept, counts, f, p, l = q.get(timeout=120)
+        results[r] = (kept, counts, f, p, l)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = W.Workload("dp", T=bounds[-1], d=32, ffn=64, E=6, k=2, act="swiglu", dtype="f32", capacity_factor=0.7,
+                    zipf_router_bias=True, seed=31, w_std=0.2)
+    full = O.route(wl, W.make_inputs(wl, with_experts=False))
+    kept_all = np.concatenate([results[r][0] for r in range(world)])
+    assert np.array_equal(kept_all, full["slot"] >= 0)
+    assert (full["slot"] < 0).any(), "the case must exercise drops"
+    for r in range(world):
+        _, counts, f, p, l = results[r]
+        assert np.array_equal(counts, full["counts"])
+        np.testing.assert_allclose(f, full["f"], rtol=1e-15)
+        np.testing.assert_allclose(p, full["p_mean"], rtol=1e-12)
+        assert abs(l - full["l_aux"]) <= 1e-12 * abs(full["l_aux"])
