@@ -68,6 +68,19 @@ typedef enum {
     MOE_ACT_GELU_BIAS = 1   /* W2( gelu_erf(x W1 + b1) ) + b2 */
 } moe_act_t;
 
+/* Router kernel.  Both compute the same logits up to fp32 summation order;
+ * each is batch-invariant (a token's logits do not depend on T or on the other
+ * tokens), and the choice never depends on T, so neither does the routing.
+ *   MOE_ROUTER_AUTO      the library's choice for the shape (currently the
+ *                        warp-MMA router);
+ *   MOE_ROUTER_WARP_MMA  warp-level mma.sync, 32-64 tokens per CTA, every dtype;
+ *   MOE_ROUTER_TCGEN05   TMA + tcgen05 tensor cores + TMEM, 128-token tiles:
+ *                        bf16, E % 8 == 0, d % 64 == 0, else
+ *                        MOE_ERR_UNSUPPORTED.
+ * Fed logits (logits_in) skip the GEMM and use the warp router's softmax and
+ * top-k whatever the choice. */
+typedef enum { MOE_ROUTER_AUTO = 0, MOE_ROUTER_WARP_MMA = 1, MOE_ROUTER_TCGEN05 = 2 } moe_router_kernel_t;
+
 /* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
  * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
 typedef struct {
@@ -80,7 +93,7 @@ typedef struct {
     int32_t act;               /* moe_act_t */
     double capacity_factor;    /* <= 0: no capacity limit (cap = T) */
     float aux_alpha;           /* alpha of L_aux */
-    int32_t reserved;          /* must be 0 */
+    int32_t router_kernel;     /* moe_router_kernel_t (0: library's choice) */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */
@@ -233,7 +246,15 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
  * launch i and stage_events[n] after the last launch, n =
  * moe_forward_launch_count(cfg) (stage_events: caller-created CUDA events,
  * at least n+1 of them).  For per-stage timing of the very same launch
- * sequence; the computation is identical to moe_forward. */
+ * sequence; the computation is identical to moe_forward.  While `stream` is
+ * being captured into a CUDA graph the events are recorded as external records
+ * (cudaEventRecordExternal), so the marks still time each replay.
+ *
+ * Graph capture: moe_forward and moe_forward_profiled make no host
+ * synchronisation and allocate nothing, so a forward on fixed buffers may be
+ * captured (after one uncaptured call on the device, which sets the kernels'
+ * attributes) and replayed; a replay reads x and the weights as they are at
+ * replay time. */
 moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
                                   const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
                                   cudaStream_t stream, cudaEvent_t* stage_events);

@@ -24,6 +24,8 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
 MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_ACT_SWIGLU, MOE_ACT_GELU_BIAS = 0, 1
+MOE_ROUTER_AUTO, MOE_ROUTER_WARP_MMA, MOE_ROUTER_TCGEN05 = 0, 1, 2
+ROUTER_KERNELS = {"auto": MOE_ROUTER_AUTO, "warp_mma": MOE_ROUTER_WARP_MMA, "tcgen05": MOE_ROUTER_TCGEN05}
 
 
 class MoEError(RuntimeError):
@@ -35,7 +37,7 @@ class MoEError(RuntimeError):
 class MoEConfigC(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("ffn", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
-                ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("reserved", ctypes.c_int32)]
+                ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("router_kernel", ctypes.c_int32)]
 
 
 class MoEWeightsC(ctypes.Structure):
@@ -114,21 +116,23 @@ class MoEConfig:
     act: str = "swiglu"        # "swiglu" | "gelu_bias"
     capacity_factor: float = 1.25
     aux_alpha: float = 0.01
+    router_kernel: str = "auto"  # "auto" | "warp_mma" | "tcgen05"
 
     def c(self) -> MoEConfigC:
         return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
                           MOE_DT_BF16 if self.dtype == "bf16" else MOE_DT_F32,
                           MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
-                          float(self.capacity_factor), float(self.aux_alpha), 0)
+                          float(self.capacity_factor), float(self.aux_alpha), ROUTER_KERNELS[self.router_kernel])
 
     @property
     def torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.dtype == "bf16" else torch.float32
 
     @staticmethod
-    def of(wl) -> "MoEConfig":
+    def of(wl, router_kernel: str = "auto") -> "MoEConfig":
         """From a workload description (anything with the same field names)."""
-        return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha)
+        return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha,
+                         router_kernel)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -310,6 +314,26 @@ class MoELayer:
 
     def forward(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None, stream=None) -> dict:
         moe_forward(self.cfg, self.weights, x, self.outputs, self.ws, logits_in, stream)
+        return self.outputs
+
+    def capture(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
+        """Records one forward on the fixed buffers `x` / `logits_in` into a CUDA
+        graph (five kernel launches, no host work when replayed).  A replay
+        reads `x` as it is at that time; results land in `self.outputs`."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(x, logits_in)  # uncaptured first call: kernel attributes, cached launch shapes
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(x, logits_in)
+        self.graph = g
+        return g
+
+    def replay(self) -> dict:
+        """Replays the graph made by `capture` on the current stream."""
+        self.graph.replay()
         return self.outputs
 
     def check(self, stream=None) -> None:

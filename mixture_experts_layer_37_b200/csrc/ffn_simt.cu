@@ -132,7 +132,7 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s) {
     p1.n_tiles = (a.ffn + TN - 1) / TN;
     cudaError_t err = swiglu ? launch_simt<S_SWIGLU>(p1, a.rows_cap, s) : launch_simt<S_GELU>(p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
-    if (a.between != nullptr && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
+    if (a.between != nullptr && (err = record_mark(a.between, s)) != cudaSuccess) return err;
     SimtParams p2;
     p2.A = static_cast<const float*>(a.h);
     p2.B0 = static_cast<const float*>(a.w2);

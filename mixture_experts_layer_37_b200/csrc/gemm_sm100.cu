@@ -349,7 +349,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     const bool pair_ok = a.rows_cap / a.E >= 512;
     cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair_ok, mA1, mB1, mB1u, p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
-    if (a.between != nullptr && (err = cudaEventRecord(a.between, s)) != cudaSuccess) return err;
+    if (a.between != nullptr && (err = record_mark(a.between, s)) != cudaSuccess) return err;
 
     GemmParams p2;
     p2.offsets = a.offsets;

@@ -44,8 +44,13 @@ struct RouterArgs {
     int fuse_scan;
     unsigned int* counter;
     ScanArgs scan;
+    DevStatus st;            // status word and wait limit (tensor-core router)
+    int kernel;              // moe_router_kernel_t
 };
 cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
+// Tensor-core router (TMA + tcgen05 + TMEM): bf16, E % 8 == 0, no logits feed.
+bool router_tc_supported(const RouterArgs& a);
+cudaError_t launch_router_tc(const RouterArgs& a, DevStatus st, cudaStream_t s);
 
 cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s);
@@ -121,5 +126,15 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_selftest_wait(DevStatus st, cudaStream_t s);
 
 int sm_count();
+
+// Records `ev` on `s`; while `s` is being captured into a CUDA graph, as an
+// external record, so that the event still marks (and times) each replay.
+inline cudaError_t record_mark(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t err = cudaStreamIsCapturing(s, &cs);
+    if (err != cudaSuccess) return err;
+    return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                                : cudaEventRecord(ev, s);
+}
 
 }  // namespace moe

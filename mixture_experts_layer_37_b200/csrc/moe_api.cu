@@ -46,7 +46,12 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->k > c->E) return MOE_ERR_INVALID_ARG;
     if (c->dtype != MOE_DT_F32 && c->dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
-    if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->reserved != 0) return MOE_ERR_INVALID_ARG;
+    if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
+        c->router_kernel > MOE_ROUTER_TCGEN05)
+        return MOE_ERR_INVALID_ARG;
+    if (c->router_kernel == MOE_ROUTER_TCGEN05 &&
+        (c->dtype != MOE_DT_BF16 || c->E % 8 != 0 || c->d % 64 != 0))
+        return MOE_ERR_UNSUPPORTED;
     if (c->E > kMaxExperts || c->k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
     if (c->T * (int64_t)c->k >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     if (c->dtype == MOE_DT_BF16) {
@@ -214,6 +219,8 @@ moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_rout
     a.fuse_scan = fused != nullptr ? 1 : 0;
     a.counter = static_cast<unsigned int*>(ws) + kStatusCounterWord;
     if (fused != nullptr) a.scan = *fused;
+    a.st = status_of(ws);
+    a.kernel = c->router_kernel;
     return from_cuda(launch_router(a, c->dtype == MOE_DT_BF16, s));
 }
 
@@ -401,7 +408,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     Plan pl;
     if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
     int n = 0;
-    auto mark = [&]() -> bool { return ev == nullptr || cudaEventRecord(ev[n++], stream) == cudaSuccess; };
+    auto mark = [&]() -> bool { return ev == nullptr || record_mark(ev[n++], stream) == cudaSuccess; };
     const ScanArgs sa = scan_args(cfg, o->counts, o->offsets, o->f, o->p, o->l_aux, true, ws, pl);
     if (cfg->T == 0) {
         // nothing to route: one launch writes the zero counts, offsets and statistics

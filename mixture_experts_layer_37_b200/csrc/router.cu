@@ -27,6 +27,7 @@
 // are added in a fixed order.  f32: one thread per token, fp32 FMA.
 #include <math.h>
 
+#include "moe.h"
 #include "scan.cuh"
 
 namespace moe {
@@ -34,7 +35,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kLStride = kMaxExperts + 1;
-constexpr int kSlabBytes = 64 * 1024;
+constexpr int kSlabBytes = 32 * 1024;  // one of the two router-weight slab buffers
 constexpr int kMaxTpc = 64;
 constexpr int kSplits = 4;  // K partial sums per token, always (batch-invariant logits)
 constexpr int kBatch = 4;  // 32-column blocks of x loaded per batch
@@ -46,6 +47,12 @@ __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
                  : "l"(p));
     return v;
 }
+
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -174,12 +181,11 @@ struct SlabGeom {
     static constexpr int kPartBytes = kSplits * kMaxTpc * 8 * NT * 4;  // [4][tpc][EP] floats
 };
 
-// Bytes of the shared region that holds the weight slab, and after the K
-// loop the K-split partial logits.
+// Bytes of the shared region that holds the two weight slab buffers, and
+// after the K loop the K-split partial logits.
 template <int NT>
 __host__ __device__ __forceinline__ int union_bytes_for(int d) {
-    const int rows = SlabGeom<NT>::kRows < d ? SlabGeom<NT>::kRows : d;
-    const int slab = (rows * SlabGeom<NT>::kPitch + 127) & ~127;
+    const int slab = d <= SlabGeom<NT>::kRows ? ((d * SlabGeom<NT>::kPitch + 127) & ~127) : 2 * kSlabBytes;
     return slab > SlabGeom<NT>::kPartBytes ? slab : SlabGeom<NT>::kPartBytes;
 }
 
@@ -230,40 +236,44 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
 #pragma unroll
         for (int n = 0; n < NT; ++n) acc[j][n][0] = acc[j][n][1] = acc[j][n][2] = acc[j][n][3] = 0.f;
 
+    // Router weight slabs: copied (cp.async, 16-byte units, no register round
+    // trip) into two alternating buffers, slab i+1 in flight while slab i is
+    // multiplied.
     const bool vec_rows = (E & 7) == 0;
-    for (int k0 = 0; k0 < d; k0 += G::kRows) {
-        const int ks = min(G::kRows, d - k0);  // multiple of 64
-        __syncthreads();
-        // stage W_r[k0 : k0+ks, :] (16-byte units, batched loads)
+    const int nslabs = (d + G::kRows - 1) / G::kRows;
+    auto stage = [&](int slab) {
+        const int k0s = slab * G::kRows;
+        const int ks = min(G::kRows, d - k0s);  // multiple of 64
+        uint8_t* dst = sW + (slab & 1) * kSlabBytes;
         const int nunits = ks * NT;
-        for (int i0 = tid; i0 < nunits; i0 += kThreads * 8) {
-            uint4 v[8];
+        for (int i = tid; i < nunits; i += kThreads) {
+            const int kk = i / NT, q = i - kk * NT;
+            uint8_t* sd = dst + slab_phys_row(kk) * G::kPitch + 16 * q;
+            if (vec_rows) {
+                cp_async_16(sd, W + (int64_t)(k0s + kk) * E + 8 * q);
+            } else {
+                __nv_bfloat16 h[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * kThreads;
-                if (i >= nunits) break;
-                const int kk = i / NT, q = i - kk * NT;
-                if (vec_rows) {
-                    v[u] = *reinterpret_cast<const uint4*>(W + (int64_t)(k0 + kk) * E + 8 * q);
-                } else {
-                    __nv_bfloat16 h[8];
-#pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const int e = 8 * q + w;
-                        h[w] = e < E ? W[(int64_t)(k0 + kk) * E + e] : __float2bfloat16(0.f);
-                    }
-                    v[u] = *reinterpret_cast<const uint4*>(h);
+                for (int w = 0; w < 8; ++w) {
+                    const int e = 8 * q + w;
+                    h[w] = e < E ? W[(int64_t)(k0s + kk) * E + e] : __float2bfloat16(0.f);
                 }
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * kThreads;
-                if (i >= nunits) break;
-                const int kk = i / NT, q = i - kk * NT;
-                *reinterpret_cast<uint4*>(sW + slab_phys_row(kk) * G::kPitch + 16 * q) = v[u];
+                *reinterpret_cast<uint4*>(sd) = *reinterpret_cast<const uint4*>(h);
             }
         }
+        cp_async_commit();
+    };
+    stage(0);
+    for (int slab = 0; slab < nslabs; ++slab) {
+        const int k0 = slab * G::kRows;
+        const int ks = min(G::kRows, d - k0);
+        if (slab + 1 < nslabs)
+            stage(slab + 1);
+        else
+            cp_async_commit();  // empty group: keeps "all but the newest group" meaning slab's copies
+        cp_async_wait_prev();
         __syncthreads();
+        const uint32_t lds_slab = lds_base + (uint32_t)((slab & 1) * kSlabBytes);
         // this warp's 32-row blocks of the slab: ksplit, ksplit + nsplit, ...
         const int nblk = ks / 32;
         for (int b0 = ksplit; b0 < nblk; b0 += nsplit * kBatch) {
@@ -285,12 +295,13 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     uint32_t b0r, b1r, b2r, b3r;
-                    ldsm_x4_trans(lds_base + (uint32_t)(32 * blk * G::kPitch + 16 * n), b0r, b1r, b2r, b3r);
+                    ldsm_x4_trans(lds_slab + (uint32_t)(32 * blk * G::kPitch + 16 * n), b0r, b1r, b2r, b3r);
                     mma_bf16_16816(acc[j][n], xa[u].x, xb[u].x, xa[u].y, xb[u].y, b0r, b1r);
                     mma_bf16_16816(acc[j][n], xa[u].z, xb[u].z, xa[u].w, xb[u].w, b2r, b3r);
                 }
             }
         }
+        __syncthreads();  // this buffer is refilled two slabs later
     }
     __syncthreads();  // the slab region is reused for the partials
 #pragma unroll
@@ -419,8 +430,15 @@ cudaError_t launch_f32_ep(RouterArgs a, cudaStream_t s) {
 
 }  // namespace
 
+// Router kernel choice: by the configuration only (never by T), so a token's
+// logits are the same whichever batch it is routed in.  The library's own
+// choice is the warp-MMA router; the tensor-core router on request.  Fed
+// logits (no GEMM to do) always take the warp router's softmax / top-k path.
+bool use_router_tc(const RouterArgs& a) { return a.kernel == MOE_ROUTER_TCGEN05 && router_tc_supported(a); }
+
 cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
+    if (bf16 && use_router_tc(a)) return launch_router_tc(a, a.st, s);
     if (bf16) {
         switch ((a.E + 7) / 8) {
             case 1: return launch_bf16_nt<1>(a, s);

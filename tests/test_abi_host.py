@@ -83,6 +83,8 @@ def test_invalid_configs_rejected_on_host(lib):
         (dict(E=0), M.MOE_ERR_INVALID_ARG),
         (dict(capacity_factor=float("nan")), M.MOE_ERR_INVALID_ARG),
         (dict(T=2 ** 30, k=2), M.MOE_ERR_UNSUPPORTED),  # T*k must stay below 2^31
+        (dict(router_kernel="tcgen05", E=12), M.MOE_ERR_UNSUPPORTED),  # tensor-core router: E % 8
+        (dict(router_kernel="tcgen05", dtype="f32", d=96), M.MOE_ERR_UNSUPPORTED),  # and bf16 only
     ]
     for kw, want in bad:
         base = dict(T=128, d=128, ffn=128, E=8, k=2)
@@ -94,6 +96,13 @@ def test_invalid_configs_rejected_on_host(lib):
     cfg = M.MoEConfig(T=8, d=128, ffn=128, E=4, k=2).c()
     cfg.dtype = 7
     assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
+    for rk in (-1, 3):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
+        cfg.router_kernel = rk
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
+    for name in ("auto", "warp_mma", "tcgen05"):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, router_kernel=name).c()
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
 
 
 def test_null_and_workspace_errors_launch_nothing(lib):

@@ -24,12 +24,16 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("wl,bounds", CASES, ids=lambda v: v.name if hasattr(v, "name") else str(len(v) - 1))
-def test_dp_shards_equal_whole_batch(wl, bounds):
+PARAMS = [(wl, b, "auto") for wl, b in CASES] + [(wl, b, "tcgen05") for wl, b in CASES if wl.E % 8 == 0]
+
+
+@pytest.mark.parametrize("wl,bounds,router", PARAMS,
+                         ids=[f"{w.name}-{len(b) - 1}-{r}" for w, b, r in PARAMS])
+def test_dp_shards_equal_whole_batch(wl, bounds, router):
     inp = W.make_inputs(wl)
     wd = weights_dev(wl, inp)
     x = to_dev(inp["x"])
-    cfg = M.MoEConfig.of(wl)
+    cfg = M.MoEConfig.of(wl, router)
     whole = M.MoELayer(cfg, wd).forward(x)
     torch.cuda.synchronize()
     world = len(bounds) - 1
@@ -37,7 +41,7 @@ def test_dp_shards_equal_whole_batch(wl, bounds):
     for r in range(world):
         t0, t1 = bounds[r], bounds[r + 1]
         c = M.MoEConfig(T=t1 - t0, d=wl.d, ffn=wl.ffn, E=wl.E, k=wl.k, dtype=wl.dtype, act=wl.act,
-                        capacity_factor=wl.capacity_factor, aux_alpha=wl.aux_alpha)
+                        capacity_factor=wl.capacity_factor, aux_alpha=wl.aux_alpha, router_kernel=router)
         o = M.allocate_outputs(c)
         o["src_assign"] = torch.empty(max(M.moe_dp_max_rows(c, wl.T), 1), dtype=torch.int32, device="cuda")
         ws = M.Workspace(c, nbytes=M.moe_dp_workspace_size(c, wl.T))

@@ -20,12 +20,12 @@ pytestmark = pytest.mark.gpu
 FULL = ["tiny_f32", "llama4moe_t4096", "flat_gelu_t8192", "longctx_zipf_t32768", "decode_t64_e64"]
 
 
-def _cfg(wl):
-    return M.MoEConfig.of(wl)
+def _cfg(wl, router="auto"):
+    return M.MoEConfig.of(wl, router)
 
 
-def _check_workload(wl, full_size: bool):
-    cfg = _cfg(wl)
+def _check_workload(wl, full_size: bool, router: str = "auto"):
+    cfg = _cfg(wl, router)
     T, E, k, d = wl.T, wl.E, wl.k, wl.d
     inp = W.make_inputs(wl)
     r = O.route(wl, inp)
@@ -53,10 +53,16 @@ def _check_workload(wl, full_size: bool):
     #         the chosen experts are the top-k of the GPU's own logits, and equal
     #         the oracle's wherever the oracle's k-th / (k+1)-th gap exceeds the bound
     lo = torch.empty((T, E), dtype=torch.float32, device="cuda")
-    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), None, idx, tw, lo, None, ws)
+    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), None, idx, tw, lo, probs, ws)
     torch.cuda.synchronize()
     lg = lo.cpu().numpy().astype(np.float64)
     gi = idx.cpu().numpy()
+    # the GPU's probabilities and weights are the softmax / renormalisation of its own logits
+    pg = probs.cpu().numpy().astype(np.float64)
+    z = np.exp(lg - lg.max(axis=1, keepdims=True))
+    assert rel_close(pg, z / z.sum(axis=1, keepdims=True), rtol=1e-5, atol=1e-12)[0]
+    sel = np.take_along_axis(pg, gi.astype(np.int64), axis=1)
+    assert rel_close(tw.cpu().numpy(), sel / sel.sum(axis=1, keepdims=True), rtol=1e-5)[0]
     toks = np.arange(T) if T <= 8192 else np.random.default_rng(1).choice(T, 8192, replace=False)
     bound = logit_error_bound(wl, inp, toks)
     err = np.abs(lg[toks] - r["logits64"][toks])
@@ -198,6 +204,17 @@ def test_benchmark_workload_parity(name):
 @pytest.mark.parametrize("wl", SMALL_WORKLOADS, ids=lambda w: w.name)
 def test_small_workload_parity(wl):
     _check_workload(wl, full_size=False)
+
+
+# the tensor-core router on every workload shape it takes (E % 8 == 0, bf16):
+# 128-token tiles with a ragged last tile, one token, E from 8 to 64
+TC_ROUTER_CASES = [w for w in SMALL_WORKLOADS if w.dtype == "bf16" and w.E % 8 == 0] + \
+    [W.WORKLOADS[n] for n in ("llama4moe_t4096", "longctx_zipf_t32768", "decode_t64_e64")]
+
+
+@pytest.mark.parametrize("wl", TC_ROUTER_CASES, ids=lambda w: w.name)
+def test_tcgen05_router_parity(wl):
+    _check_workload(wl, full_size=wl.T > 4096, router="tcgen05")
 
 
 def test_empty_batch():
