@@ -25,7 +25,8 @@
  *   - Every tensor pointer is DEVICE memory owned by the caller, row-major,
  *     contiguous, 16-byte aligned, unless the comment says HOST.  The
  *     library never allocates or frees memory and never synchronises, except
- *     in moe_check_device_status (which synchronises the given stream).
+ *     in moe_check_device_status (which synchronises the given stream) and
+ *     in the moe_pipeline_* object, which owns its buffers and streams.
  *   - "act" tensors (x, x_perm, h, y_perm, out and the weights) have the
  *     config's dtype: float32 (MOE_DT_F32) or bfloat16 (MOE_DT_BF16).
  *     Router logits, probabilities, top-k weights, f, p and L_aux are float32;
@@ -274,6 +275,50 @@ moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* we
  * check (`*site`, if not NULL, receives the code of the first wait that gave
  * up), MOE_ERR_CUDA if the synchronisation failed, else MOE_OK. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t* site);
+
+/* ---- Pipelined forwards on host-resident batches ------------------------
+ * A stream of layer forwards whose inputs and outputs live in HOST memory
+ * (pinned, e.g. cudaHostAlloc, for the copies to run asynchronously).  Step i
+ * copies its batch in, runs moe_forward on it and copies the layer output and
+ * L_aux back; the copy in of step i+1, the forward of step i and the copy out
+ * of step i-1 run at the same time (three streams; `depth` device buffer
+ * slots for x and out).  Each step's results are those of moe_forward on the
+ * same batch, bit for bit.  The object allocates its device buffers, workspace
+ * and routing outputs with cudaMalloc on the current device at creation and
+ * frees them in moe_pipeline_destroy; `weights` (device, caller-owned) must
+ * stay valid and unchanged until then.  Not thread-safe: one host thread at a
+ * time per pipeline. */
+#define MOE_PIPELINE_MAX_DEPTH 4
+typedef struct moe_pipeline moe_pipeline_t;
+
+/* depth: 1..MOE_PIPELINE_MAX_DEPTH slots (2 overlaps copy in, forward and
+ * copy out).  *pipe receives the object, or NULL on error.  Returns
+ * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED for a bad config, weights or
+ * depth (nothing allocated), MOE_ERR_CUDA if an allocation or stream creation
+ * failed (everything released). */
+moe_status_t moe_pipeline_create(const moe_config_t* cfg, const moe_weights_t* weights, int32_t depth,
+                                 moe_pipeline_t** pipe);
+
+/* Queues one step: x_host (HOST, [T,d] config dtype) -> forward ->
+ * out_host (HOST, [T,d]) and l_aux_host (HOST, 1 float).  Returns without
+ * waiting; x_host must not change and out_host / l_aux_host must not be read
+ * until moe_pipeline_wait(ticket) returns.  start_event (if not NULL) is
+ * recorded just before the copy in, end_event (if not NULL) just after the
+ * copy out, for device-side timing.  *ticket (if not NULL) receives the
+ * step's number (0, 1, ...). */
+moe_status_t moe_pipeline_submit(moe_pipeline_t* pipe, const void* x_host, void* out_host, float* l_aux_host,
+                                 cudaEvent_t start_event, cudaEvent_t end_event, int64_t* ticket);
+
+/* Blocks until step `ticket`'s results are in host memory (ticket < 0: every
+ * submitted step).  MOE_ERR_INVALID_ARG for a ticket not yet submitted. */
+moe_status_t moe_pipeline_wait(moe_pipeline_t* pipe, int64_t ticket);
+
+/* moe_check_device_status on the pipeline's workspace (synchronises its
+ * compute stream). */
+moe_status_t moe_pipeline_check(moe_pipeline_t* pipe, uint32_t* site);
+
+/* Waits for every queued step, then frees everything the object holds. */
+moe_status_t moe_pipeline_destroy(moe_pipeline_t* pipe);
 
 /* Time limit of every bounded device wait, in milliseconds (default 2000).
  * Applies to launches made after the call; process-wide. */

@@ -101,7 +101,8 @@ EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_wo
                     "moe_forward", "moe_forward_hostio", "moe_check_device_status", "moe_set_wait_timeout_ms",
                     "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled",
                     "moe_dispatch_noalloc", "moe_dp_workspace_size", "moe_dp_max_rows", "moe_dp_route",
-                    "moe_dp_finish")
+                    "moe_dp_finish", "moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_wait",
+                    "moe_pipeline_check", "moe_pipeline_destroy")
 
 
 # ---------------------------------------------------------------- config
@@ -399,3 +400,65 @@ def moe_dp_finish(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: in
     oc = _outputs_c(outputs)
     _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank),
              ctypes.byref(wc), _ptr(x), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_finish")
+
+
+# ---------------------------------------------------------------- pipelined forwards on host batches
+class Pipeline:
+    """moe_pipeline_*: forwards on host-resident batches, the copy in of the
+    next batch and the copy out of the previous one overlapping the current
+    forward.  Host tensors should be pinned (``pin_memory()``); they must stay
+    untouched (inputs) or unread (outputs) until ``wait`` covers their step."""
+
+    def __init__(self, cfg: MoEConfig, weights: dict, depth: int = 2):
+        L = lib()
+        L.moe_pipeline_create.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), ctypes.c_int32, ctypes.POINTER(_P)]
+        L.moe_pipeline_submit.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.POINTER(ctypes.c_int64)]
+        L.moe_pipeline_wait.argtypes = [_P, ctypes.c_int64]
+        L.moe_pipeline_check.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_pipeline_destroy.argtypes = [_P]
+        for n in ("moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_wait", "moe_pipeline_check",
+                  "moe_pipeline_destroy"):
+            getattr(L, n).restype = ctypes.c_int
+        self._L = L
+        self.cfg = cfg
+        self.weights = weights  # kept alive: the pipeline reads them on every step
+        self._wc = _weights_c(weights)
+        h = _P()
+        _check(L.moe_pipeline_create(ctypes.byref(cfg.c()), ctypes.byref(self._wc), int(depth), ctypes.byref(h)),
+               "moe_pipeline_create")
+        self._h = h
+
+    def submit(self, x_host: torch.Tensor, out_host: torch.Tensor, l_aux_host: torch.Tensor,
+               start_event=None, end_event=None) -> int:
+        t = ctypes.c_int64()
+        _check(self._L.moe_pipeline_submit(self._h, _ptr(x_host), _ptr(out_host), _ptr(l_aux_host),
+                                           start_event.cuda_event if start_event is not None else None,
+                                           end_event.cuda_event if end_event is not None else None,
+                                           ctypes.byref(t)), "moe_pipeline_submit")
+        return t.value
+
+    def wait(self, ticket: int = -1) -> None:
+        _check(self._L.moe_pipeline_wait(self._h, int(ticket)), "moe_pipeline_wait")
+
+    def check(self) -> None:
+        site = ctypes.c_uint32()
+        st = self._L.moe_pipeline_check(self._h, ctypes.byref(site))
+        if st != MOE_OK:
+            raise MoEError(st, f"pipeline device status (site 0x{site.value:x})")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _check(self._L.moe_pipeline_destroy(self._h), "moe_pipeline_destroy")
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -152,3 +152,30 @@ def test_status_strings(lib):
     for s in range(6):
         assert M.moe_status_string(s).startswith("MOE_")
     assert "UNKNOWN" in M.moe_status_string(99)
+
+
+def test_pipeline_arguments_checked_before_any_cuda_call(lib):
+    """moe_pipeline_* refuse bad arguments on the host (no GPU needed)."""
+    P = ctypes.c_void_p
+    lib.moe_pipeline_create.argtypes = [ctypes.POINTER(M.MoEConfigC), ctypes.POINTER(M.MoEWeightsC), ctypes.c_int32,
+                                        ctypes.POINTER(P)]
+    lib.moe_pipeline_submit.argtypes = [P, P, P, P, P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.moe_pipeline_wait.argtypes = [P, ctypes.c_int64]
+    lib.moe_pipeline_check.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.moe_pipeline_destroy.argtypes = [P]
+    cfg = M.MoEConfig(T=128, d=128, ffn=128, E=8, k=2).c()
+    w = M.MoEWeightsC(16, None, 32, 48, 64, None, None)  # never dereferenced on the host
+    h = P()
+    assert lib.moe_pipeline_create(ctypes.byref(cfg), ctypes.byref(w), 2, None) == M.MOE_ERR_INVALID_ARG
+    for depth in (0, 5, -1):
+        assert lib.moe_pipeline_create(ctypes.byref(cfg), ctypes.byref(w), depth, ctypes.byref(h)) == \
+            M.MOE_ERR_INVALID_ARG
+        assert h.value is None
+    bad = M.MoEConfig(T=128, d=100, ffn=128, E=8, k=2).c()
+    assert lib.moe_pipeline_create(ctypes.byref(bad), ctypes.byref(w), 2, ctypes.byref(h)) == M.MOE_ERR_UNSUPPORTED
+    now = M.MoEWeightsC(None, None, 32, 48, 64, None, None)
+    assert lib.moe_pipeline_create(ctypes.byref(cfg), ctypes.byref(now), 2, ctypes.byref(h)) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_submit(None, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_wait(None, -1) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_check(None, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_destroy(None) == M.MOE_ERR_INVALID_ARG
