@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router-kernel", default="auto", choices=["auto", "warp_mma", "tcgen05"])
+    ap.add_argument("--gemm-kernel", default="auto", choices=["auto", "one_cta", "cta_pair"])
     return ap.parse_args()
 
 
@@ -180,7 +182,7 @@ def run_native(a):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     wl = W.WORKLOADS[a.workload]
-    cfg = M.MoEConfig.of(wl)
+    cfg = M.MoEConfig.of(wl, a.router_kernel, a.gemm_kernel)
     seed = wl.seed + 1000 * rank
     inp = W.make_inputs(wl, seed=seed)
 
@@ -385,7 +387,8 @@ def run_native(a):
                    "act": wl.act, "capacity_factor": wl.capacity_factor, "rows_dispatched": R,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
-                   "launch": "timed steps replayed from one captured CUDA graph"},
+                   "launch": "timed steps replayed from one captured CUDA graph",
+                   "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel},
         "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * a.steps,
         "clocks": clocks, "cpu_baseline": cpu,
     }

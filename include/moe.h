@@ -82,6 +82,16 @@ typedef enum {
  * top-k whatever the choice. */
 typedef enum { MOE_ROUTER_AUTO = 0, MOE_ROUTER_WARP_MMA = 1, MOE_ROUTER_TCGEN05 = 2 } moe_router_kernel_t;
 
+/* Expert GEMM kernel (bf16; the f32 path has one kernel).  Same results bit
+ * for bit: every output element is one fp32 tensor-core sum over K in the
+ * same order, rounded once.
+ *   MOE_GEMM_AUTO      the library's choice per GEMM;
+ *   MOE_GEMM_ONE_CTA   one CTA per 128-row tile (M=128, N=256);
+ *   MOE_GEMM_CTA_PAIR  two CTAs per 256-row tile (tcgen05 cta_group::2), an
+ *                      expert's last tile as a 128-row pair tile when it holds
+ *                      at most 128 rows. */
+typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_ONE_CTA = 1, MOE_GEMM_CTA_PAIR = 2 } moe_gemm_kernel_t;
+
 /* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
  * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
 typedef struct {
@@ -95,6 +105,8 @@ typedef struct {
     double capacity_factor;    /* <= 0: no capacity limit (cap = T) */
     float aux_alpha;           /* alpha of L_aux */
     int32_t router_kernel;     /* moe_router_kernel_t (0: library's choice) */
+    int32_t gemm_kernel;       /* moe_gemm_kernel_t (0: library's choice) */
+    int32_t reserved;          /* must be 0 */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */

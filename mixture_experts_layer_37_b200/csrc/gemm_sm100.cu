@@ -33,6 +33,7 @@
 // Every wait is bounded in time; on expiry the kernel records a timeout,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "gemm_common.cuh"
+#include "moe.h"
 
 namespace moe {
 namespace {
@@ -295,24 +296,13 @@ cudaError_t launch_pair_gemm(int mode, const CUtensorMap& a, const CUtensorMap& 
 
 namespace {
 // Kernel choice per GEMM.  The CTA pair halves the weight bytes each SM loads
-// and reads per MMA, but pads each expert's rows to 256 instead of 128.  It is
-// used for the second GEMM and for the GELU first GEMM (long K per tile or a
-// heavy epilogue), and when an expert is expected to hold at least 512 rows;
-// the one-CTA kernel for the SwiGLU first GEMM and for small batches.
-// MOE_GEMM_CTA_PAIR=0/1 forces one kernel (benchmarking).
-int forced_variant() {
-    static int v = -2;
-    if (v == -2) {
-        const char* env = getenv("MOE_GEMM_CTA_PAIR");
-        v = env == nullptr ? -1 : (env[0] == '0' ? 0 : 1);
-    }
-    return v;
-}
-
-cudaError_t launch_one(int mode, bool pair_ok, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+// and reads per MMA; an expert's rows are padded to a multiple of 128 by
+// either kernel (the pair runs a last tile of at most 128 rows as an M=128
+// pair tile).  The library's choice: the pair when an expert is expected to
+// hold at least 512 rows, else the one-CTA kernel, whose 128-row tiles give
+// more independent tiles to spread over the SMs.
+cudaError_t launch_one(int mode, bool pair, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int64_t rows_cap, cudaStream_t s) {
-    const int f = forced_variant();
-    const bool pair = f >= 0 ? f == 1 : (pair_ok && mode != MODE_SWIGLU);
     if (pair) return launch_pair_gemm(mode, a, b0, b1, p, rows_cap, s);
     if (mode == MODE_SWIGLU) return launch_mode<MODE_SWIGLU>(a, b0, b1, p, rows_cap, s);
     if (mode == MODE_GELU) return launch_mode<MODE_GELU>(a, b0, b1, p, rows_cap, s);
@@ -346,8 +336,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p1.n_tiles = (a.ffn + p1.bn_out - 1) / p1.bn_out;
     p1.st = a.st;
     // rows an expert is expected to receive (the routing itself stays on the device)
-    const bool pair_ok = a.rows_cap / a.E >= 512;
-    cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair_ok, mA1, mB1, mB1u, p1, a.rows_cap, s);
+    const bool pair = a.gemm_kernel == MOE_GEMM_CTA_PAIR || (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512);
+    cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair, mA1, mB1, mB1u, p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
     if (a.between != nullptr && (err = record_mark(a.between, s)) != cudaSuccess) return err;
 
@@ -361,7 +351,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p2.bn_out = 256;
     p2.n_tiles = (a.d + 255) / 256;
     p2.st = a.st;
-    return launch_one(MODE_PLAIN, pair_ok, mA2, mB2, mB2, p2, a.rows_cap, s);
+    return launch_one(MODE_PLAIN, pair, mA2, mB2, mB2, p2, a.rows_cap, s);
 }
 
 }  // namespace moe

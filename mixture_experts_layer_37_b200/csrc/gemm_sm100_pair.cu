@@ -19,8 +19,15 @@
 //     on the `empty` / `tfull` barrier at the same offset in both CTAs.
 //   - Accumulator free: each epilogue warp of both CTAs arrives on the
 //     leader's `tempty` barrier (8 arrivals).
-// SwiGLU: CTA 0 loads the gate columns and CTA 1 the up columns of the
-// tile's 128 output columns, so each CTA's accumulator rows hold [gate | up].
+// An expert's last tile, when it holds at most 128 rows, runs as an M=128
+// pair tile instead (64 rows per CTA), which halves its padding: each CTA's
+// accumulator then holds its 64 rows twice over, TMEM lanes 0-63 for the
+// first 128 of the 256 columns and lanes 64-127 for the other 128, in TMEM
+// columns 0-127 (the two-CTA M=128 data-path layout).
+// Column order of the 256 accumulator columns: CTA 0's 128 weight columns
+// first, then CTA 1's.  SwiGLU: CTA r loads the gate and the up box of output
+// columns [64r, 64r+64) of the tile's 128, so every 128-column half holds
+// [gate 64 | up 64] of the same 64 outputs, in both tile shapes.
 // Every wait is bounded in time, as in the one-CTA kernel.
 #include "gemm_common.cuh"
 
@@ -36,6 +43,80 @@ constexpr int kBStageP = 2 * kBBoxBytes;         // 16 KB: this CTA's 128 of the
 constexpr int kStageP = kAStageP + kBStageP;     // 32 KB
 constexpr int kSmemP = kStagesP * kStageP + 1024 + kBiasBytes + 1024;
 constexpr uint32_t kIdescP = make_idesc(BMP, BN_MMA);
+constexpr uint32_t kIdescPHalf = make_idesc(BMP / 2, BN_MMA);
+
+// Epilogue of one warp for `ncols` accumulator columns starting at TMEM column
+// offset 0 of `tbase`, written to output columns [out0, out0 + ncols) (SwiGLU:
+// ncols/2 outputs from [gate 64 | up 64] groups).  `wb` is the warp's bias
+// staging row.  Warp-collective.
+template <int MODE>
+__device__ __forceinline__ void epilogue_pair(const GemmParams& p, uint32_t tbase, __nv_bfloat16* orow, bool valid,
+                                              int out0, int ncols, int e, __nv_bfloat16* wb, int lane) {
+    if (MODE == MODE_SWIGLU) {
+        for (int g = 0; g < ncols; g += 128) {
+            const int o = out0 + g / 2;
+#pragma unroll 1
+            for (int c = 0; c < 64; c += 16) {
+                uint32_t gv[16], uv[16];
+                tmem_ld_16(tbase + g + c, gv);
+                tmem_ld_16(tbase + g + 64 + c, uv);
+                tmem_ld_wait();
+                if (valid && o + c < p.N) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float h0 = silu_f(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+                        const float h1 = silu_f(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
+                        pk[i] = pack_bf16x2(h0, h1);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(orow + o + c);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+        }
+    } else {
+        if (p.bias != nullptr) {
+            __syncwarp();
+            const int col = out0 + 8 * lane;
+            uint4 bv = make_uint4(0, 0, 0, 0);
+            if (8 * lane < ncols && col < p.N) bv = *reinterpret_cast<const uint4*>(p.bias + (int64_t)e * p.N + col);
+            reinterpret_cast<uint4*>(wb)[lane] = bv;
+            __syncwarp();
+        }
+#pragma unroll 1
+        for (int c = 0; c < ncols; c += 16) {
+            uint32_t v[16];
+            tmem_ld_16(tbase + c, v);
+            tmem_ld_wait();
+            if (valid && out0 + c < p.N) {
+                float x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(v[i]);
+                if (p.bias != nullptr) {
+                    const uint4* b4 = reinterpret_cast<const uint4*>(wb + c);
+                    const uint4 bA = b4[0], bB = b4[1];
+                    const uint32_t bw[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        x[2 * i] += bf16_lo(bw[i]);
+                        x[2 * i + 1] += bf16_hi(bw[i]);
+                    }
+                }
+                if (MODE == MODE_GELU) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = gelu_f(x[i]);
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+                uint4* dst = reinterpret_cast<uint4*>(orow + out0 + c);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        }
+    }
+}
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -109,8 +190,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int tile = pair; tile < total_tiles && !stop; tile += npairs) {
                 int e, row0, rows, nt;
                 decode_tile(tile, mt_prefix, s_off, p.n_tiles, BMP, e, row0, rows, nt);
-                const CUtensorMap* mb = (MODE == MODE_SWIGLU && rank == 1) ? &tmB1 : &tmB0;
-                const int col0 = (MODE == MODE_SWIGLU) ? nt * 128 : nt * 256 + 128 * (int)rank;
+                // this CTA's rows: 128 of a full tile, 64 of a half (M=128) tile
+                const int arow = row0 + (rows <= BMP / 2 ? 64 : 128) * (int)rank;
+                const int col0 = (MODE == MODE_SWIGLU) ? nt * 128 + 64 * (int)rank : nt * 256 + 128 * (int)rank;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (*abort_flag) { stop = true; break; }
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, tmo)) {
@@ -122,10 +204,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t bar = full_lead + 8u * stage;
                     uint8_t* a_dst = sA + stage * kAStageP;
                     uint8_t* b_dst = sB + stage * kBStageP;
-                    tma_load_2d_pair(a_dst, &tmA, bar, kb * BK, row0 + 128 * (int)rank);
+                    tma_load_2d_pair(a_dst, &tmA, bar, kb * BK, arow);
                     const int krow = e * p.K + kb * BK;
-                    tma_load_2d_pair(b_dst, mb, bar, col0, krow);
-                    tma_load_2d_pair(b_dst + kBBoxBytes, mb, bar, col0 + 64, krow);
+                    if (MODE == MODE_SWIGLU) {
+                        tma_load_2d_pair(b_dst, &tmB0, bar, col0, krow);                // gate
+                        tma_load_2d_pair(b_dst + kBBoxBytes, &tmB1, bar, col0, krow);   // up
+                    } else {
+                        tma_load_2d_pair(b_dst, &tmB0, bar, col0, krow);
+                        tma_load_2d_pair(b_dst + kBBoxBytes, &tmB0, bar, col0 + 64, krow);
+                    }
                     issued_mask |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStagesP) {
@@ -149,6 +236,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool stop = false;
             for (int tile = pair; tile < total_tiles && !stop; tile += npairs) {
+                int e, row0, rows, nt;
+                decode_tile(tile, mt_prefix, s_off, p.n_tiles, BMP, e, row0, rows, nt);
+                const uint32_t idesc = rows <= BMP / 2 ? kIdescPHalf : kIdescP;
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, tmo)) {
                     give_up(SITE_GEMM_MMA_TMEM_EMPTY);
                     break;
@@ -169,7 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
-                        tc_mma_f16_pair(d_tmem, adesc, bdesc, kIdescP, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);
                     if (++stage == kStagesP) {
@@ -205,11 +295,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int r = 128 * (int)rank + q * 32 + lane;
+            // full tile: this warp's 32 of the CTA's 128 rows, all 256 columns;
+            // half tile: rows 32(q&1).. of the CTA's 64, columns [128(q>>1), +128)
+            const bool half = rows <= BMP / 2;
+            const int r = half ? 64 * (int)rank + 32 * (q & 1) + lane : 128 * (int)rank + q * 32 + lane;
+            const int ncols = half ? 128 : 256;
+            const int out0 = nt * p.bn_out + (half ? (q >> 1) * (MODE == MODE_SWIGLU ? 64 : 128) : 0);
             const bool valid = r < rows;
             __nv_bfloat16* orow = p.out + (int64_t)(row0 + (valid ? r : 0)) * p.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
-            epilogue_rows<MODE>(p, tbase, orow, valid, nt * p.bn_out, e, wb, lane);
+            epilogue_pair<MODE>(p, tbase, orow, valid, out0, ncols, e, wb, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * acc);

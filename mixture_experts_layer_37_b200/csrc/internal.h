@@ -116,6 +116,7 @@ struct FfnArgs {
     const void* b2;          // [E, d] or null
     DevStatus st;
     cudaEvent_t between;     // recorded between the two GEMM launches, or null
+    int gemm_kernel;         // moe_gemm_kernel_t
 };
 // bf16: tcgen05 grouped GEMMs (two launches).  Returns cudaErrorInvalidValue
 // when a tensor map cannot be encoded.

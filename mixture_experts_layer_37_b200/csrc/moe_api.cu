@@ -47,7 +47,8 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->dtype != MOE_DT_F32 && c->dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
-        c->router_kernel > MOE_ROUTER_TCGEN05)
+        c->router_kernel > MOE_ROUTER_TCGEN05 || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
+        c->reserved != 0)
         return MOE_ERR_INVALID_ARG;
     if (c->router_kernel == MOE_ROUTER_TCGEN05 &&
         (c->dtype != MOE_DT_BF16 || c->E % 8 != 0 || c->d % 64 != 0))
@@ -264,6 +265,7 @@ moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* 
     f.b2 = w->b2;
     f.st = status_of(ws);
     f.between = between;
+    f.gemm_kernel = c->gemm_kernel;
     return from_cuda(c->dtype == MOE_DT_BF16 ? launch_ffn_bf16_sm100(f, s) : launch_ffn_f32(f, s));
 }
 

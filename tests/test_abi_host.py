@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_config_struct_layout_matches_header():
-    assert ctypes.sizeof(M.MoEConfigC) == 48
+    assert ctypes.sizeof(M.MoEConfigC) == 56
     assert M.MoEConfigC.capacity_factor.offset == 32
     assert ctypes.sizeof(M.MoEWeightsC) == 7 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
 
@@ -103,6 +103,13 @@ def test_invalid_configs_rejected_on_host(lib):
     for name in ("auto", "warp_mma", "tcgen05"):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, router_kernel=name).c()
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
+    for name in ("auto", "one_cta", "cta_pair"):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, gemm_kernel=name).c()
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
+    for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("reserved", 1)):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
+        setattr(cfg, field, v)
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
 
 
 def test_null_and_workspace_errors_launch_nothing(lib):

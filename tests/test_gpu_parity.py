@@ -20,12 +20,12 @@ pytestmark = pytest.mark.gpu
 FULL = ["tiny_f32", "llama4moe_t4096", "flat_gelu_t8192", "longctx_zipf_t32768", "decode_t64_e64"]
 
 
-def _cfg(wl, router="auto"):
-    return M.MoEConfig.of(wl, router)
+def _cfg(wl, router="auto", gemm="auto"):
+    return M.MoEConfig.of(wl, router, gemm)
 
 
-def _check_workload(wl, full_size: bool, router: str = "auto"):
-    cfg = _cfg(wl, router)
+def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto"):
+    cfg = _cfg(wl, router, gemm)
     T, E, k, d = wl.T, wl.E, wl.k, wl.d
     inp = W.make_inputs(wl)
     r = O.route(wl, inp)
@@ -215,6 +215,43 @@ TC_ROUTER_CASES = [w for w in SMALL_WORKLOADS if w.dtype == "bf16" and w.E % 8 =
 @pytest.mark.parametrize("wl", TC_ROUTER_CASES, ids=lambda w: w.name)
 def test_tcgen05_router_parity(wl):
     _check_workload(wl, full_size=wl.T > 4096, router="tcgen05")
+
+
+# both expert-GEMM kernels on every bf16 shape: ragged experts, drops, one
+# expert, k = E, a single token, 16 experts; the pair kernel's 128-row tail
+# tiles appear wherever an expert's rows end within 128 of a 256 boundary
+GEMM_CASES = [(w, g) for w in SMALL_WORKLOADS if w.dtype == "bf16" for g in ("one_cta", "cta_pair")] + \
+    [(W.WORKLOADS["llama4moe_t4096"], "cta_pair"), (W.WORKLOADS["llama4moe_t4096"], "one_cta"),
+     (W.WORKLOADS["flat_gelu_t8192"], "one_cta"), (W.WORKLOADS["decode_t64_e64"], "cta_pair")]
+
+
+@pytest.mark.parametrize("wl,gemm", GEMM_CASES, ids=[f"{w.name}-{g}" for w, g in GEMM_CASES])
+def test_gemm_kernel_parity(wl, gemm):
+    _check_workload(wl, full_size=wl.T > 4096, gemm=gemm)
+
+
+@pytest.mark.parametrize("wl", [w for w in SMALL_WORKLOADS if w.dtype == "bf16"] + [W.WORKLOADS["llama4moe_t4096"]],
+                         ids=lambda w: w.name)
+def test_gemm_kernels_agree_bitwise(wl):
+    """The one-CTA and the CTA-pair kernels give the same bits: each output is
+    the same fp32 tensor-core sum over K, rounded once."""
+    inp = W.make_inputs(wl)
+    r = O.route(wl, inp)
+    wd = weights_dev(wl, inp)
+    R = int(r["offsets"][-1])
+    outs = []
+    for g in ("one_cta", "cta_pair"):
+        cfg = _cfg(wl, gemm=g)
+        rows_cap = M.moe_max_rows(cfg)
+        xperm = np.zeros((max(rows_cap, 1), wl.d), dtype=inp["x"].dtype)
+        xperm[:R] = inp["x"][r["src_assign"] // wl.k]
+        y = torch.zeros((max(rows_cap, 1), wl.d), dtype=cfg.torch_dtype, device="cuda")
+        ws = M.Workspace(cfg)
+        M.moe_expert_ffn(cfg, wd, to_dev(xperm), to_dev(r["offsets"]), y, ws)
+        torch.cuda.synchronize()
+        assert M.moe_check_device_status(ws)[0] == M.MOE_OK
+        outs.append(y[:R].cpu())
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
 
 
 def test_empty_batch():
