@@ -29,7 +29,9 @@
 // Tiles walk the ragged per-expert row groups: the tile list (m-tiles per
 // expert) is built on the device from the kept-row offsets, so the host never
 // reads the routing result.  A tile that runs past its expert's last row
-// reads the next rows (or TMA zero-fill) and masks them at the store.
+// reads the next rows (or TMA zero-fill) and masks them at the store; an
+// expert's last tile of at most 64 rows runs as an M=64 MMA (half the work),
+// whose accumulator rows sit in lanes 0-15 of each 32-lane TMEM quarter.
 // Every wait is bounded in time; on expiry the kernel records a timeout,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "gemm_common.cuh"
@@ -47,6 +49,7 @@ constexpr int kBStageBytes = 4 * kBBoxBytes;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;   // 48 KB
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + 1024 /*alignment*/;
 constexpr uint32_t kIdesc = make_idesc(BM, BN_MMA);
+constexpr uint32_t kIdesc64 = make_idesc(BM / 2, BN_MMA);
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -160,6 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool stop = false;
             for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+                int e, row0, rows, nt;
+                decode_tile(tile, mt_prefix, s_off, p.n_tiles, BM, e, row0, rows, nt);
+                const uint32_t idesc = rows <= BM / 2 ? kIdesc64 : kIdesc;
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, tmo)) {
                     give_up(SITE_GEMM_MMA_TMEM_EMPTY);
                     break;
@@ -183,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         //    64-column boxes are 8 KB apart (leading byte offset).
                         const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, kBBoxBytes, 1024);
-                        tc_mma_f16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -217,8 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int r = q * 32 + lane;
-            const bool valid = r < rows;
+            // M=128: row 32q + lane.  M=64 (a last tile of at most 64 rows):
+            // rows 16q..16q+15 sit in lanes 0-15 of this warp's quarter
+            const bool m64 = rows <= BM / 2;
+            const int r = m64 ? 16 * q + lane : q * 32 + lane;
+            const bool valid = r < rows && (!m64 || lane < 16);
             __nv_bfloat16* orow = p.out + (int64_t)(row0 + (valid ? r : 0)) * p.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
             epilogue_rows<MODE>(p, tbase, orow, valid, nt * p.bn_out, e, wb, lane);
