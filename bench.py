@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-kernel", default="auto", choices=["auto", "warp_mma", "tcgen05"])
     ap.add_argument("--gemm-kernel", default="auto", choices=["auto", "one_cta", "cta_pair"])
+    ap.add_argument("--dispatch", default="auto", choices=["auto", "copy", "gather"])
     return ap.parse_args()
 
 
@@ -182,7 +183,7 @@ def run_native(a):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     wl = W.WORKLOADS[a.workload]
-    cfg = M.MoEConfig.of(wl, a.router_kernel, a.gemm_kernel)
+    cfg = M.MoEConfig.of(wl, a.router_kernel, a.gemm_kernel, a.dispatch)
     seed = wl.seed + 1000 * rank
     inp = W.make_inputs(wl, seed=seed)
 
@@ -388,7 +389,7 @@ def run_native(a):
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
                    "launch": "timed steps replayed from one captured CUDA graph",
-                   "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel},
+                   "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel, "dispatch": a.dispatch},
         "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * a.steps,
         "clocks": clocks, "cpu_baseline": cpu,
     }

@@ -92,6 +92,20 @@ typedef enum { MOE_ROUTER_AUTO = 0, MOE_ROUTER_WARP_MMA = 1, MOE_ROUTER_TCGEN05 
  *                      at most 128 rows. */
 typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_ONE_CTA = 1, MOE_GEMM_CTA_PAIR = 2 } moe_gemm_kernel_t;
 
+/* How the first expert GEMM of moe_forward / moe_dp_finish gets its rows
+ * (bf16; the f32 path always copies).  Same results bit for bit.
+ *   MOE_DISPATCH_AUTO    the library's choice (currently COPY: the gathering
+ *                        producer's 16-byte copies keep the tensor cores
+ *                        waiting, so its first GEMM is slower than copy plus
+ *                        TMA tiles);
+ *   MOE_DISPATCH_COPY    the dispatch kernel copies each kept row to the
+ *                        expert-sorted x_perm, which the GEMM reads by TMA;
+ *   MOE_DISPATCH_GATHER  the GEMM's producer warp gathers the token rows of x
+ *                        straight into its shared-memory tiles (one-CTA
+ *                        kernel); the dispatch kernel writes only slot and
+ *                        src_assign, and x_perm is never written. */
+typedef enum { MOE_DISPATCH_AUTO = 0, MOE_DISPATCH_COPY = 1, MOE_DISPATCH_GATHER = 2 } moe_dispatch_mode_t;
+
 /* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
  * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
 typedef struct {
@@ -106,7 +120,7 @@ typedef struct {
     float aux_alpha;           /* alpha of L_aux */
     int32_t router_kernel;     /* moe_router_kernel_t (0: library's choice) */
     int32_t gemm_kernel;       /* moe_gemm_kernel_t (0: library's choice) */
-    int32_t reserved;          /* must be 0 */
+    int32_t dispatch;          /* moe_dispatch_mode_t (0: library's choice) */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */

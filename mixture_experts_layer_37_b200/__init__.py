@@ -28,6 +28,8 @@ MOE_ROUTER_AUTO, MOE_ROUTER_WARP_MMA, MOE_ROUTER_TCGEN05 = 0, 1, 2
 ROUTER_KERNELS = {"auto": MOE_ROUTER_AUTO, "warp_mma": MOE_ROUTER_WARP_MMA, "tcgen05": MOE_ROUTER_TCGEN05}
 MOE_GEMM_AUTO, MOE_GEMM_ONE_CTA, MOE_GEMM_CTA_PAIR = 0, 1, 2
 GEMM_KERNELS = {"auto": MOE_GEMM_AUTO, "one_cta": MOE_GEMM_ONE_CTA, "cta_pair": MOE_GEMM_CTA_PAIR}
+MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER = 0, 1, 2
+DISPATCH_MODES = {"auto": MOE_DISPATCH_AUTO, "copy": MOE_DISPATCH_COPY, "gather": MOE_DISPATCH_GATHER}
 
 
 class MoEError(RuntimeError):
@@ -40,7 +42,7 @@ class MoEConfigC(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("ffn", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("router_kernel", ctypes.c_int32),
-                ("gemm_kernel", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("gemm_kernel", ctypes.c_int32), ("dispatch", ctypes.c_int32)]
 
 
 class MoEWeightsC(ctypes.Structure):
@@ -122,23 +124,24 @@ class MoEConfig:
     aux_alpha: float = 0.01
     router_kernel: str = "auto"  # "auto" | "warp_mma" | "tcgen05"
     gemm_kernel: str = "auto"    # "auto" | "one_cta" | "cta_pair"
+    dispatch: str = "auto"       # "auto" | "copy" | "gather"
 
     def c(self) -> MoEConfigC:
         return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
                           MOE_DT_BF16 if self.dtype == "bf16" else MOE_DT_F32,
                           MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
                           float(self.capacity_factor), float(self.aux_alpha), ROUTER_KERNELS[self.router_kernel],
-                          GEMM_KERNELS[self.gemm_kernel], 0)
+                          GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch])
 
     @property
     def torch_dtype(self) -> torch.dtype:
         return torch.bfloat16 if self.dtype == "bf16" else torch.float32
 
     @staticmethod
-    def of(wl, router_kernel: str = "auto", gemm_kernel: str = "auto") -> "MoEConfig":
+    def of(wl, router_kernel: str = "auto", gemm_kernel: str = "auto", dispatch: str = "auto") -> "MoEConfig":
         """From a workload description (anything with the same field names)."""
         return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha,
-                         router_kernel, gemm_kernel)
+                         router_kernel, gemm_kernel, dispatch)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

@@ -109,6 +109,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, uin
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only), and an arrival on
+// `bar` once all of this thread's earlier cp.async copies have landed (the
+// arrival counts toward the barrier's expected count: .noinc).
+__device__ __forceinline__ void cp_async_16_cg(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }

@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
         }
     }
     if (tid < nA) a.slot[a_base + tid] = s;
+    if (a.x_perm == nullptr) return;  // rows gathered by the first GEMM instead
     sSlot[tid] = s;
     __syncthreads();
     // row gather: each warp copies two rows at a time (16-byte vectors, up to

@@ -46,6 +46,11 @@ struct GemmParams {
     int bn_out;                  // output columns per tile: 128 (SwiGLU) or 256
     int n_tiles;
     DevStatus st;
+    // A rows gathered from the token activations instead of a sorted copy:
+    // row s of the expert-sorted order is token src_assign[s] / k of gx
+    const __nv_bfloat16* gx;     // [T, K] or null (A read through its tensor map)
+    const int32_t* src_assign;   // [R]
+    int k;
 };
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }

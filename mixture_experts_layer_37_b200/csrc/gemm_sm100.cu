@@ -47,11 +47,13 @@ constexpr int kStages = 4;
 constexpr int kAStageBytes = BM * BK * 2;                  // 16 KB
 constexpr int kBStageBytes = 4 * kBBoxBytes;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;   // 48 KB
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + 1024 /*alignment*/;
+constexpr int kTokBytes = BM * 4;                          // gathered tile: token of each row
+constexpr int kSmemBytes =
+    kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + kTokBytes + 1024 /*alignment*/;
 constexpr uint32_t kIdesc = make_idesc(BM, BN_MMA);
 constexpr uint32_t kIdesc64 = make_idesc(BM / 2, BN_MMA);
 
-template <int MODE>
+template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, GemmParams p) {
@@ -70,12 +72,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* mt_prefix = reinterpret_cast<int*>(tmem_slot + 2);   // [E+1]
     int* s_off = mt_prefix + (kMaxExperts + 1);                // [E+1]
     __nv_bfloat16* s_bias = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes + 1024);  // [4][256]
+    int* s_tok = reinterpret_cast<int*>(smem + kStages * kStageBytes + 1024 + kBiasBytes);           // [BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            // gathered A: the 32 producer lanes' cp.async arrivals join the TMA's
+            mbar_init(&full[s], GATHER ? 33 : 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&tfull[0], 1);
@@ -108,7 +112,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
     };
 
-    if (warp == 0) {
+    if (warp == 0 && GATHER) {
+        // ------------------------------------------------ gathering producer (whole warp)
+        // A tile: lane L copies 16-byte chunk L % 8 of rows L / 8 + 4i of the
+        // tile straight from the token rows (8 lanes read one row's 128 bytes),
+        // to the place the 128-byte swizzle gives it; B as in the TMA producer.
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued_mask = 0, issued_par = 0;
+        bool stop = false;
+        const int R = s_off[p.E];
+        const int ch = lane & 7;
+        for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+            int e, row0, rows, nt;
+            decode_tile(tile, mt_prefix, s_off, p.n_tiles, BM, e, row0, rows, nt);
+            const int n0 = nt * p.bn_out;
+            __syncwarp();  // every lane is done with the previous tile's tokens
+            for (int r = lane; r < BM; r += 32) {
+                const int row = row0 + r;
+                s_tok[r] = row < R ? p.src_assign[row] / p.k : 0;  // rows past R: any valid row, masked later
+            }
+            __syncwarp();
+            for (int kb = 0; kb < kblocks; ++kb) {
+                if (__shfl_sync(0xffffffffu, *abort_flag, 0)) { stop = true; break; }
+                const bool free_ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, tmo);
+                if (!__all_sync(0xffffffffu, free_ok)) {
+                    if (lane == 0) give_up(SITE_GEMM_PRODUCER_EMPTY);
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[stage], kBStageBytes);
+                    uint8_t* b_dst = sB + stage * kBStageBytes;
+                    const int krow = e * p.K + kb * BK;
+                    if (MODE == MODE_SWIGLU) {
+                        tma_load_2d(b_dst, &tmB0, &full[stage], n0, krow);
+                        tma_load_2d(b_dst + kBBoxBytes, &tmB0, &full[stage], n0 + 64, krow);
+                        tma_load_2d(b_dst + 2 * kBBoxBytes, &tmB1, &full[stage], n0, krow);
+                        tma_load_2d(b_dst + 3 * kBBoxBytes, &tmB1, &full[stage], n0 + 64, krow);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            tma_load_2d(b_dst + i * kBBoxBytes, &tmB0, &full[stage], n0 + 64 * i, krow);
+                    }
+                }
+                uint8_t* a_dst = sA + stage * kAStageBytes;
+                const __nv_bfloat16* gsrc = p.gx + kb * BK + ch * 8;
+#pragma unroll 8
+                for (int i = 0; i < BM / 4; ++i) {
+                    const int r = (lane >> 3) + 4 * i;
+                    cp_async_16_cg(a_dst + r * 128 + ((ch ^ (r & 7)) << 4), gsrc + (int64_t)s_tok[r] * p.K);
+                }
+                cp_async_mbar_arrive_noinc(&full[stage]);
+                issued_mask |= 1u << stage;
+                issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // no copy may still be landing in shared memory when the CTA exits
+        if (lane == 0)
+            for (int s = 0; s < kStages; ++s)
+                if ((issued_mask >> s) & 1u)
+                    if (!mbar_wait_bounded(&full[s], (issued_par >> s) & 1u, tmo)) give_up(SITE_GEMM_PRODUCER_DRAIN);
+    } else if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
             int stage = 0;
@@ -180,6 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
+                    // gathered A was written by cp.async (generic proxy); the MMA reads it through the async proxy
+                    if (GATHER) fence_proxy_async_smem();
                     const uint32_t a_addr = smem_u32(sA + stage * kAStageBytes);
                     const uint32_t b_addr = smem_u32(sB + stage * kBStageBytes);
 #pragma unroll
@@ -263,22 +334,22 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int MODE>
+template <int MODE, bool GATHER = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                         int64_t rows_cap, cudaStream_t s) {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t err =
-            cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, GATHER>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (err != cudaSuccess) return err;
         if (dev < 64) attr_set[dev] = true;
     }
     const int64_t tiles_upper = (rows_cap / BM + p.E) * (int64_t)p.n_tiles;
     const int grid = (int)min64(tiles_upper, (int64_t)sm_count());
     if (grid <= 0) return cudaSuccess;
-    grouped_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
+    grouped_gemm_kernel<MODE, GATHER><<<grid, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
     return cudaGetLastError();
 }
 
@@ -312,6 +383,10 @@ namespace {
 // more independent tiles to spread over the SMs.
 cudaError_t launch_one(int mode, bool pair, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int64_t rows_cap, cudaStream_t s) {
+    if (p.gx != nullptr) {  // first GEMM with its rows gathered from the tokens (one-CTA kernel)
+        if (mode == MODE_SWIGLU) return launch_mode<MODE_SWIGLU, true>(a, b0, b1, p, rows_cap, s);
+        return launch_mode<MODE_GELU, true>(a, b0, b1, p, rows_cap, s);
+    }
     if (pair) return launch_pair_gemm(mode, a, b0, b1, p, rows_cap, s);
     if (mode == MODE_SWIGLU) return launch_mode<MODE_SWIGLU>(a, b0, b1, p, rows_cap, s);
     if (mode == MODE_GELU) return launch_mode<MODE_GELU>(a, b0, b1, p, rows_cap, s);
@@ -344,6 +419,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p1.bn_out = swiglu ? 128 : 256;
     p1.n_tiles = (a.ffn + p1.bn_out - 1) / p1.bn_out;
     p1.st = a.st;
+    p1.gx = static_cast<const __nv_bfloat16*>(a.gather_x);
+    p1.src_assign = a.src_assign;
+    p1.k = a.k;
     // rows an expert is expected to receive (the routing itself stays on the device)
     const bool pair = a.gemm_kernel == MOE_GEMM_CTA_PAIR || (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512);
     cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair, mA1, mB1, mB1u, p1, a.rows_cap, s);
@@ -360,6 +438,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p2.bn_out = 256;
     p2.n_tiles = (a.d + 255) / 256;
     p2.st = a.st;
+    p2.gx = nullptr;
+    p2.src_assign = nullptr;
+    p2.k = a.k;
     return launch_one(MODE_PLAIN, pair, mA2, mB2, mB2, p2, a.rows_cap, s);
 }
 

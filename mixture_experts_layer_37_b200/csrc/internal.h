@@ -62,7 +62,7 @@ struct ScatterArgs {
     int32_t* slot;              // [T, k]
     int32_t* src_assign;        // [R_max]
     const void* x;              // [T, d]
-    void* x_perm;               // [R_max, d]
+    void* x_perm;               // [R_max, d], or null: no row copies (slot / src_assign only)
     const int32_t* cap_e;       // [E] per-expert capacity left for this batch, or null (use cap)
     int64_t T;
     int E, k, cap, nchunk;
@@ -117,6 +117,11 @@ struct FfnArgs {
     DevStatus st;
     cudaEvent_t between;     // recorded between the two GEMM launches, or null
     int gemm_kernel;         // moe_gemm_kernel_t
+    // when gather_x != null the first GEMM reads its rows straight from the
+    // tokens (row s = token src_assign[s] / k) and x_perm is not used
+    const void* gather_x;    // [T, d] or null
+    const int32_t* src_assign;
+    int k;
 };
 // bf16: tcgen05 grouped GEMMs (two launches).  Returns cudaErrorInvalidValue
 // when a tensor map cannot be encoded.

@@ -48,7 +48,7 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
         c->router_kernel > MOE_ROUTER_TCGEN05 || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
-        c->reserved != 0)
+        c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER)
         return MOE_ERR_INVALID_ARG;
     if (c->router_kernel == MOE_ROUTER_TCGEN05 &&
         (c->dtype != MOE_DT_BF16 || c->E % 8 != 0 || c->d % 64 != 0))
@@ -246,8 +246,13 @@ moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* id
     return from_cuda(launch_dispatch_scatter(xa, s));
 }
 
+// Whether moe_forward / moe_dp_finish gather the first GEMM's rows from x
+// (on request only: the copy is faster end to end on B200).
+bool gathers(const moe_config_t* c) { return c->dtype == MOE_DT_BF16 && c->dispatch == MOE_DISPATCH_GATHER; }
+
 moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* x_perm, const int32_t* offsets,
-                     void* y_perm, void* ws, const Plan& pl, cudaStream_t s, cudaEvent_t between = nullptr) {
+                     void* y_perm, void* ws, const Plan& pl, cudaStream_t s, cudaEvent_t between = nullptr,
+                     const void* gather_x = nullptr, const int32_t* src_assign = nullptr) {
     FfnArgs f;
     f.act = c->act;
     f.E = c->E;
@@ -266,6 +271,9 @@ moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* 
     f.st = status_of(ws);
     f.between = between;
     f.gemm_kernel = c->gemm_kernel;
+    f.gather_x = gather_x;
+    f.src_assign = src_assign;
+    f.k = c->k;
     return from_cuda(c->dtype == MOE_DT_BF16 ? launch_ffn_bf16_sm100(f, s) : launch_ffn_f32(f, s));
 }
 
@@ -425,10 +433,13 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
                     o->logits_out, o->probs_out, ws, pl, stream, &sa);
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, x_perm, ws, pl, stream);
+    const bool gather = gathers(cfg);
+    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
+                     stream);
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr);
+    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr,
+                 gather ? x : nullptr, o->src_assign);
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
     st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
@@ -525,9 +536,12 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
     if (cfg->T == 0) return MOE_OK;
     void* x_perm = at(ws, pl.xperm);
     void* y_perm = at(ws, pl.yperm);
-    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, x_perm, ws, pl, stream, dp.cap_e);
+    const bool gather = gathers(cfg);
+    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
+                     stream, dp.cap_e);
     if (st != MOE_OK) return st;
-    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream);
+    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, nullptr, gather ? x : nullptr,
+                 o->src_assign);
     if (st != MOE_OK) return st;
     return run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
 }

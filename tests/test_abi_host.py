@@ -106,7 +106,10 @@ def test_invalid_configs_rejected_on_host(lib):
     for name in ("auto", "one_cta", "cta_pair"):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, gemm_kernel=name).c()
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
-    for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("reserved", 1)):
+    for name in ("auto", "copy", "gather"):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, dispatch=name).c()
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
+    for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("dispatch", 3), ("dispatch", -1)):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
         setattr(cfg, field, v)
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG

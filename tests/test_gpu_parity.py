@@ -301,3 +301,31 @@ def test_bounded_wait_gives_up_and_context_survives():
     layer.check()
     ref = O.forward(wl, inp, routing=r)
     assert out_close(host_f64(o["out"]), ref["out"], "bf16")[0]
+
+
+# the first expert GEMM reading its rows straight from x (gather) against the
+# expert-sorted copy: every forward output bit for bit
+DISPATCH_CASES = [w for w in SMALL_WORKLOADS if w.dtype == "bf16"] + \
+    [W.WORKLOADS[n] for n in ("llama4moe_t4096", "longctx_zipf_t32768", "decode_t64_e64", "flat_gelu_t8192")]
+
+
+@pytest.mark.parametrize("wl", DISPATCH_CASES, ids=lambda w: w.name)
+def test_gather_dispatch_equals_copy(wl):
+    inp = W.make_inputs(wl)
+    wd = weights_dev(wl, inp)
+    x = to_dev(inp["x"])
+    outs = {}
+    for mode in ("copy", "gather"):
+        for gemm in ("one_cta", "cta_pair"):
+            layer = M.MoELayer(M.MoEConfig.of(wl, gemm_kernel=gemm, dispatch=mode), wd)
+            o = layer.forward(x)
+            layer.check()
+            outs[(mode, gemm)] = {n: v.clone() for n, v in o.items()}
+    ref = outs[("copy", "one_cta")]
+    R = int(ref["offsets"][-1])
+    for key, o in outs.items():
+        for n, v in ref.items():
+            a, b = v, o[n]
+            if n == "src_assign":
+                a, b = a[:R], b[:R]
+            assert torch.equal(a, b), f"{key}: {n} differs"
