@@ -149,9 +149,16 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- native
+GEMM_SOURCES = ("gemm_sm100.cu", "gemm_sm100_pair.cu", "gemm_common.cuh", "common.cuh")
+
+
 def kernel_source_hash() -> str:
-    p = os.path.join(ROOT, "mixture_experts_layer_37_b200", "csrc", "gemm_sm100.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    """Hash of the grouped-GEMM sources; recorded ncu traffic is used only while it matches."""
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "mixture_experts_layer_37_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):

@@ -376,11 +376,13 @@ cudaError_t launch_pair_gemm(int mode, const CUtensorMap& a, const CUtensorMap& 
 
 namespace {
 // Kernel choice per GEMM.  The CTA pair halves the weight bytes each SM loads
-// and reads per MMA; an expert's rows are padded to a multiple of 128 by
-// either kernel (the pair runs a last tile of at most 128 rows as an M=128
-// pair tile).  The library's choice: the pair when an expert is expected to
-// hold at least 512 rows, else the one-CTA kernel, whose 128-row tiles give
-// more independent tiles to spread over the SMs.
+// and reads per MMA, and its 256-row tiles halve the number of tiles; an
+// expert's rows are padded to a multiple of 128 by either kernel (the pair
+// runs a last tile of at most 128 rows as an M=128 pair tile).  The library's
+// choice, from same-machine measurements of both kernels on every benchmark
+// workload: the one-CTA kernel for the first GEMM (the pair was 1-7 % slower
+// there), and the pair for the second GEMM when an expert is expected to hold
+// at least 512 rows (its long-K tiles come in fewer, fuller waves).
 cudaError_t launch_one(int mode, bool pair, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int64_t rows_cap, cudaStream_t s) {
     if (p.gx != nullptr) {  // first GEMM with its rows gathered from the tokens (one-CTA kernel)
@@ -423,8 +425,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p1.src_assign = a.src_assign;
     p1.k = a.k;
     // rows an expert is expected to receive (the routing itself stays on the device)
-    const bool pair = a.gemm_kernel == MOE_GEMM_CTA_PAIR || (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512);
-    cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair, mA1, mB1, mB1u, p1, a.rows_cap, s);
+    const bool pair1 = a.gemm_kernel == MOE_GEMM_CTA_PAIR;
+    const bool pair2 = a.gemm_kernel == MOE_GEMM_CTA_PAIR || (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512);
+    cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair1, mA1, mB1, mB1u, p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
     if (a.between != nullptr && (err = record_mark(a.between, s)) != cudaSuccess) return err;
 
@@ -441,7 +444,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p2.gx = nullptr;
     p2.src_assign = nullptr;
     p2.k = a.k;
-    return launch_one(MODE_PLAIN, pair, mA2, mB2, mB2, p2, a.rows_cap, s);
+    return launch_one(MODE_PLAIN, pair2, mA2, mB2, mB2, p2, a.rows_cap, s);
 }
 
 }  // namespace moe
