@@ -34,6 +34,15 @@ DESIGN.md):
       are rounded to fp32 before selection, and softmax uses those values.
   R6  GELU is the exact erf form (PyTorch nn.GELU() default).
   R7  T = 0: nothing is routed; f = p = 0 and L_aux = 0.
+  R16 padding tokens ([LLaMA4-MoE] §4.1: padding is kept out of expert
+      selection): a token with token_mask = 0 selects no expert (index -1,
+      weight 0, no dispatch, no routed output) and is left out of f and p,
+      which divide by the number of real tokens T_real; the capacity stays
+      ceil(T*k/E * cf) of the whole batch T.  T_real = 0 gives zero statistics.
+  R17 shared experts ([LLaMA4-MoE] §5.2: fixed experts take part in every
+      token's computation): n_shared experts of the routed experts' form, own
+      weights, applied to every token (padding included) with weight 1 and
+      added after the routed terms: out[t] = sum_j w[t,j] y(t,j) + sum_s y_s(t).
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py
 (worked example, closed forms, brute force, invariants, library
@@ -134,7 +143,7 @@ def dispatch(idx: np.ndarray, E: int, cap: int) -> dict:
     """
     T, k = idx.shape
     flat = idx.reshape(-1).astype(np.int64)
-    rank = np.empty(T * k, dtype=np.int64)
+    rank = np.full(T * k, np.iinfo(np.int64).max, dtype=np.int64)  # index -1 (padding, R16): never kept
     counts = np.zeros(E, dtype=np.int64)
     for e in range(E):
         pos = np.nonzero(flat == e)[0]          # ascending assignment order = token-major
@@ -143,7 +152,7 @@ def dispatch(idx: np.ndarray, E: int, cap: int) -> dict:
     kept = np.minimum(counts, cap)
     offsets = np.zeros(E + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(kept)
-    keep = rank < cap
+    keep = (flat >= 0) & (rank < cap)
     slot = np.where(keep, offsets[flat] + rank, -1)
     src_assign = np.empty(int(offsets[-1]), dtype=np.int64)
     src_assign[slot[keep]] = np.nonzero(keep)[0]
@@ -200,6 +209,26 @@ def combine(y_by_assignment: dict, slot: np.ndarray, w: np.ndarray, T: int, d: i
     return out
 
 
+def mask_padding(idx: np.ndarray, w: np.ndarray, token_mask: Optional[np.ndarray]) -> tuple:
+    """Reading R16: a padding token (token_mask = 0) selects no expert: its
+    indices become -1 and its weights 0 ([LLaMA4-MoE] §4.1)."""
+    if token_mask is None:
+        return idx, w
+    pad = np.asarray(token_mask) == 0
+    idx = idx.copy()
+    w = w.copy()
+    idx[pad] = -1
+    w[pad] = 0.0
+    return idx, w
+
+
+def real_tokens(token_mask: Optional[np.ndarray], T: int) -> np.ndarray:
+    """Reading R16: the tokens that count in f and p (all of them without a mask)."""
+    if token_mask is None:
+        return np.ones(T, dtype=bool)
+    return np.asarray(token_mask) != 0
+
+
 def aux_stats(counts: np.ndarray, p: np.ndarray, T: int, k: int, alpha: float) -> tuple:
     """Load-balance statistics ([MoE-basics] §2.3 and §3.1; [LLaMA4-MoE] §3.2):
     f_e = n_e / (T*k) (reading R4), p_e = mean over tokens of the full softmax,
@@ -219,7 +248,8 @@ def route(wl, inputs: dict, logits_feed: Optional[np.ndarray] = None) -> dict:
     """Router, softmax, top-k, renormalisation, capacity dispatch and aux stats
     over all T tokens.  ``logits_feed`` (float32 [T,E]) replaces the router
     product when both sides must take the discrete decisions on identical
-    logits; it must come from this oracle or from the input generator."""
+    logits; it must come from this oracle or from the input generator.
+    ``inputs['token_mask']`` (uint8 [T], optional) marks padding (R16)."""
     T, E, k = wl.T, wl.E, wl.k
     if logits_feed is None:
         x = to_f64(inputs["x"], wl.dtype)
@@ -231,11 +261,14 @@ def route(wl, inputs: dict, logits_feed: Optional[np.ndarray] = None) -> dict:
     p = softmax(l) if T > 0 else np.zeros((0, E))
     idx = select_topk(l, k) if T > 0 else np.zeros((0, k), dtype=np.int32)
     w = renormalise(p, idx) if T > 0 else np.zeros((0, k))
+    mask = inputs.get("token_mask")
+    idx, w = mask_padding(idx, w, mask)
     cap = capacity(T, k, E, wl.capacity_factor)
     disp = dispatch(idx, E, cap)
-    f, pm, laux = aux_stats(disp["counts"], p, T, k, wl.aux_alpha)
+    real = real_tokens(mask, T)
+    f, pm, laux = aux_stats(disp["counts"], p[real], int(real.sum()), k, wl.aux_alpha)
     return {"logits64": l64, "logits": l, "p": p, "idx": idx, "w": w, "cap": cap,
-            "f": f, "p_mean": pm, "l_aux": laux, **disp}
+            "f": f, "p_mean": pm, "l_aux": laux, "t_real": int(real.sum()), **disp}
 
 
 def expert_weights_f64(wl, inputs: dict, e: int) -> tuple:
@@ -245,6 +278,16 @@ def expert_weights_f64(wl, inputs: dict, e: int) -> tuple:
         return (to_f64(inputs["w_gate"][e], dt), to_f64(inputs["w_up"][e], dt), to_f64(inputs["w_down"][e], dt))
     return (to_f64(inputs["w1"][e], dt), to_f64(inputs["b1"][e], dt),
             to_f64(inputs["w2"][e], dt), to_f64(inputs["b2"][e], dt))
+
+
+def shared_weights_f64(wl, inputs: dict, s: int) -> tuple:
+    """Shared expert s's parameters decoded to float64 (reading R17)."""
+    dt = wl.dtype
+    if wl.act == "swiglu":
+        return (to_f64(inputs["shared_gate"][s], dt), to_f64(inputs["shared_up"][s], dt),
+                to_f64(inputs["shared_down"][s], dt))
+    return (to_f64(inputs["shared_w1"][s], dt), to_f64(inputs["shared_b1"][s], dt),
+            to_f64(inputs["shared_w2"][s], dt), to_f64(inputs["shared_b2"][s], dt))
 
 
 def expert_apply(wl, params: tuple, xr: np.ndarray) -> np.ndarray:
@@ -293,4 +336,20 @@ def forward(wl, inputs: dict, logits_feed: Optional[np.ndarray] = None,
     assigns = np.array([t * k + j for t in toks for j in range(k)], dtype=np.int64)
     y = expert_outputs(wl, inputs, r, assigns, x_rows)
     out = combine(y, r["slot"], r["w"], T, wl.d, toks)
+    n_shared = getattr(wl, "n_shared", 0)
+    if n_shared > 0 and toks.size > 0:
+        if x_rows is not None:
+            xr = np.stack([x_rows[int(t)] for t in toks])
+        else:
+            xr = to_f64(inputs["x"][toks], wl.dtype)
+        out = out + shared_outputs(wl, inputs, xr)
     return {**r, "out": out, "tokens": toks, "y": y}
+
+
+def shared_outputs(wl, inputs: dict, xr: np.ndarray) -> np.ndarray:
+    """Reading R17: the sum over the shared experts (in order, weight 1 each) of
+    their outputs on rows ``xr`` ([LLaMA4-MoE] §5.2)."""
+    acc = np.zeros((xr.shape[0], wl.d), dtype=np.float64)
+    for s_ in range(wl.n_shared):
+        acc = acc + expert_apply(wl, shared_weights_f64(wl, inputs, s_), xr)
+    return acc

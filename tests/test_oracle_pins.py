@@ -351,11 +351,85 @@ def check_empty(o):
     assert r["src_assign"].size == 0
 
 
+def check_padding_mask(o):
+    """Reading R16 (padding kept out of expert selection, LLaMA4-MoE page §4.1):
+    an all-ones mask changes nothing; with no capacity limit, the real tokens of
+    a padded batch route exactly as the batch of real tokens alone, with the
+    same statistics; padding selects nothing and outputs 0; padding does not use
+    capacity (hand case); an all-padding batch has zero statistics."""
+    wl = _wl(T=24, d=8, ffn=12, E=4, k=2, capacity_factor=0.0)
+    inp = W.make_inputs(wl.with_(seed=11))
+    base = o.route(wl, inp)
+    ones = o.route(wl, {**inp, "token_mask": np.ones(wl.T, dtype=np.uint8)})
+    for key in ("idx", "w", "counts", "offsets", "slot", "f", "p_mean"):
+        np.testing.assert_array_equal(base[key], ones[key])
+    mask = np.ones(wl.T, dtype=np.uint8)
+    pad = np.array([0, 3, 4, 10, 17, 23])
+    mask[pad] = 0
+    real = np.nonzero(mask)[0]
+    masked = o.forward(wl, {**inp, "token_mask": mask})
+    wl_r = wl.with_(T=real.size)
+    alone = o.forward(wl_r, {**inp, "x": inp["x"][real]})
+    np.testing.assert_array_equal(masked["idx"][real], alone["idx"])
+    np.testing.assert_allclose(masked["w"][real], alone["w"], rtol=0, atol=0)
+    np.testing.assert_array_equal(masked["counts"], alone["counts"])
+    np.testing.assert_allclose(masked["f"], alone["f"], rtol=1e-15)
+    np.testing.assert_allclose(masked["p_mean"], alone["p_mean"], rtol=1e-13)
+    assert abs(masked["l_aux"] - alone["l_aux"]) <= 1e-15
+    assert (masked["idx"][pad] == -1).all() and (masked["w"][pad] == 0).all() and (masked["slot"][pad] == -1).all()
+    np.testing.assert_allclose(masked["out"][real], alone["out"], rtol=1e-13, atol=1e-15)
+    assert (masked["out"][pad] == 0).all()
+    # hand case: T=4, E=1, k=1, cf=0.5 -> cap 2; token 0 is padding, so tokens 1, 2 are kept, 3 dropped
+    wl1 = _wl(T=4, d=8, ffn=12, E=1, k=1, capacity_factor=0.5)
+    inp1 = W.make_inputs(wl1.with_(seed=3))
+    r1 = o.route(wl1, {**inp1, "token_mask": np.array([0, 1, 1, 1], dtype=np.uint8)})
+    assert r1["slot"][:, 0].tolist() == [-1, 0, 1, -1] and r1["counts"].tolist() == [3]
+    assert abs(r1["f"][0] - 1.0) < 1e-15
+    # every token padding
+    r0 = o.route(wl, {**inp, "token_mask": np.zeros(wl.T, dtype=np.uint8)})
+    assert (r0["counts"] == 0).all() and (r0["f"] == 0).all() and (r0["p_mean"] == 0).all() and r0["l_aux"] == 0.0
+    assert r0["offsets"][-1] == 0
+
+
+def check_shared_experts(o):
+    """Reading R17 (shared experts in every token's computation, LLaMA4-MoE
+    page §5.2): with one routed expert (E=1, k=1, no limit) and one shared
+    expert the layer is the sum of two textbook dense FFNs; two identical shared
+    experts add twice one; padding tokens get the shared output only."""
+    import torch
+    for act in ("swiglu", "gelu_bias"):
+        wl = _wl(T=21, d=16, ffn=24, E=1, k=1, act=act, capacity_factor=0.0, n_shared=1)
+        inp = _dense_inputs(act, T=21)
+        sh = _dense_inputs(act, T=21, seed=9)
+        keys = ("w_gate", "w_up", "w_down") if act == "swiglu" else ("w1", "b1", "w2", "b2")
+        shared = {"shared_" + {"w_gate": "gate", "w_up": "up", "w_down": "down"}.get(k_, k_): sh[k_] for k_ in keys}
+        res = o.forward(wl, {**inp, **shared})
+        x = torch.from_numpy(inp["x"].astype(np.float64))
+
+        def ffn(params):
+            if act == "swiglu":
+                g = x @ torch.from_numpy(params["w_gate"][0].astype(np.float64))
+                u = x @ torch.from_numpy(params["w_up"][0].astype(np.float64))
+                return (torch.nn.functional.silu(g) * u) @ torch.from_numpy(params["w_down"][0].astype(np.float64))
+            h = torch.nn.functional.gelu(x @ torch.from_numpy(params["w1"][0].astype(np.float64))
+                                         + torch.from_numpy(params["b1"][0].astype(np.float64)))
+            return h @ torch.from_numpy(params["w2"][0].astype(np.float64)) + torch.from_numpy(params["b2"][0].astype(np.float64))
+
+        ref = ffn(inp) + ffn(sh)
+        np.testing.assert_allclose(res["out"], ref.numpy(), rtol=1e-12, atol=1e-12)
+        two = {k_: np.concatenate([v, v]) for k_, v in shared.items()}
+        res2 = o.forward(wl.with_(n_shared=2), {**inp, **two})
+        np.testing.assert_allclose(res2["out"] - res["out"], ffn(sh).numpy(), rtol=1e-12, atol=1e-12)
+        pad = o.forward(wl, {**inp, **shared, "token_mask": np.zeros(21, dtype=np.uint8)})
+        np.testing.assert_allclose(pad["out"], ffn(sh).numpy(), rtol=1e-12, atol=1e-12)
+
+
 CHECKS = [check_worked_example, check_uniform_alpha, check_sums_to_one, check_topk_bruteforce,
           check_tie_lower_id, check_renorm_is_selected_softmax, check_softmax_closed_form,
           check_capacity, check_dispatch_hand_case, check_dispatch_bruteforce,
           check_activation_closed_forms, check_dense_reduction, check_teaching_layer,
-          check_combine_properties, check_drop_path_end_to_end, check_empty]
+          check_combine_properties, check_drop_path_end_to_end, check_empty, check_padding_mask,
+          check_shared_experts]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
@@ -445,7 +519,25 @@ def _swiglu_swapped(xr, wg, wu, wd):
     return np.matmul(O.silu(np.matmul(xr, wu)) * np.matmul(xr, wg), wd)
 
 
+def _mask_ignored(idx, w, token_mask):
+    return idx, w
+
+
+def _stats_over_all_tokens(token_mask, T):
+    return np.ones(T, dtype=bool)
+
+
+def _shared_averaged(wl, inputs, xr):
+    acc = np.zeros((xr.shape[0], wl.d))
+    for s_ in range(wl.n_shared):
+        acc = acc + O.expert_apply(wl, O.shared_weights_f64(wl, inputs, s_), xr)
+    return acc / max(wl.n_shared, 1)
+
+
 MUTANTS = {
+    "padding_selects_experts": dict(mask_padding=_mask_ignored),
+    "padding_counted_in_stats": dict(real_tokens=_stats_over_all_tokens),
+    "shared_experts_averaged": dict(shared_outputs=_shared_averaged),
     "tie_upper_id": dict(select_topk=_topk_upper_tie),
     "capacity_without_k": dict(capacity=_cap_without_k),
     "f_divided_by_T": dict(aux_stats=_aux_f_over_T),

@@ -30,6 +30,8 @@ _lib = None
 
 # stream ids of the generator, one per tensor
 STREAM_X, STREAM_WR, STREAM_W1, STREAM_WUP, STREAM_W2, STREAM_B1, STREAM_B2 = 1, 2, 3, 4, 5, 6, 7
+# shared experts' parameters and the padding draw
+STREAM_SW1, STREAM_SWUP, STREAM_SW2, STREAM_SB1, STREAM_SB2, STREAM_PAD = 8, 9, 10, 11, 12, 13
 
 
 def build_generator(force: bool = False) -> str:
@@ -103,6 +105,8 @@ class Workload:
     w_std: float = 0.02
     b_std: float = 0.01
     seed: int = 0
+    n_shared: int = 0         # always-on shared experts (same FFN form as the routed ones)
+    pad_fraction: float = 0.0  # expected fraction of padding tokens (token_mask = 0)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -138,9 +142,33 @@ def make_inputs(wl: Workload, seed: Optional[int] = None, with_experts: bool = T
         "w_router": normal(s, STREAM_WR, (wl.d, wl.E), wl.w_std, dt),
         "router_bias": zipf_bias(wl.E) if wl.zipf_router_bias else None,
     }
+    if wl.pad_fraction > 0:
+        # token t is padding when its uniform draw falls below pad_fraction
+        out["token_mask"] = (uniform_f64(s, STREAM_PAD, wl.T) >= wl.pad_fraction).astype(np.uint8)
     if with_experts:
         out.update(make_expert_weights(wl, s))
+        if wl.n_shared > 0:
+            out.update(make_shared_weights(wl, s))
     return out
+
+
+def make_shared_weights(wl: Workload, seed: Optional[int] = None) -> dict:
+    """Parameters of the n_shared always-on experts, same shapes per expert as the routed ones."""
+    s = wl.seed if seed is None else seed
+    dt = wl.dtype
+    S, d, F = wl.n_shared, wl.d, wl.ffn
+    if wl.act == "swiglu":
+        return {
+            "shared_gate": normal(s, STREAM_SW1, (S, d, F), wl.w_std, dt),
+            "shared_up": normal(s, STREAM_SWUP, (S, d, F), wl.w_std, dt),
+            "shared_down": normal(s, STREAM_SW2, (S, F, d), wl.w_std, dt),
+        }
+    return {
+        "shared_w1": normal(s, STREAM_SW1, (S, d, F), wl.w_std, dt),
+        "shared_b1": normal(s, STREAM_SB1, (S, F), wl.b_std, dt),
+        "shared_w2": normal(s, STREAM_SW2, (S, F, d), wl.w_std, dt),
+        "shared_b2": normal(s, STREAM_SB2, (S, d), wl.b_std, dt),
+    }
 
 
 def make_expert_weights(wl: Workload, seed: Optional[int] = None) -> dict:
