@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--router-kernel", default="auto", choices=["auto", "warp_mma", "tcgen05"])
     ap.add_argument("--gemm-kernel", default="auto", choices=["auto", "one_cta", "cta_pair"])
     ap.add_argument("--dispatch", default="auto", choices=["auto", "copy", "gather"])
+    ap.add_argument("--n-shared", type=int, default=None, help="shared experts (default: the workload's)")
+    ap.add_argument("--pad-fraction", type=float, default=None, help="padding tokens (default: the workload's)")
     return ap.parse_args()
 
 
@@ -190,6 +192,10 @@ def run_native(a):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     wl = W.WORKLOADS[a.workload]
+    if a.n_shared is not None:
+        wl = wl.with_(n_shared=a.n_shared)
+    if a.pad_fraction is not None:
+        wl = wl.with_(pad_fraction=a.pad_fraction)
     cfg = M.MoEConfig.of(wl, a.router_kernel, a.gemm_kernel, a.dispatch)
     seed = wl.seed + 1000 * rank
     inp = W.make_inputs(wl, seed=seed)
@@ -199,10 +205,13 @@ def run_native(a):
             return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
         return torch.from_numpy(np.ascontiguousarray(arr)).cuda()
 
-    weights = {n: dev(inp[n]) for n in ("w_router", "w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2") if n in inp}
+    wnames = ("w_router", "w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2", "shared_gate", "shared_up",
+              "shared_down", "shared_w1", "shared_b1", "shared_w2", "shared_b2")
+    weights = {n: dev(inp[n]) for n in wnames if n in inp}
     if inp.get("router_bias") is not None:
         weights["router_bias"] = dev(np.asarray(inp["router_bias"], dtype=np.float32))
     x = dev(inp["x"])
+    tmask = dev(inp["token_mask"]) if "token_mask" in inp else None
     layer = M.MoELayer(cfg, weights)
     nl = M.moe_forward_launch_count(cfg)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -224,7 +233,7 @@ def run_native(a):
 
     for _ in range(a.warmup):
         clear_l2()
-        layer.forward(x)
+        layer.forward(x, token_mask=tmask)
     torch.cuda.synchronize()
     layer.check()
 
@@ -233,7 +242,7 @@ def run_native(a):
     torch.cuda.synchronize()
     for i in range(a.steps):
         clear_l2()
-        M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, eager[i])
+        M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, eager[i], token_mask=tmask)
     torch.cuda.synchronize()
     eager_ms = float(sum(ev[0].elapsed_time(ev[nl]) for ev in eager))
 
@@ -244,7 +253,7 @@ def run_native(a):
     with torch.cuda.graph(graph):
         for i in range(a.steps):
             clear_l2()
-            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, steps[i])
+            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, steps[i], token_mask=tmask)
     graph.replay()  # upload and warm the graph
     torch.cuda.synchronize()
     layer.check()
@@ -274,7 +283,9 @@ def run_native(a):
 
     # ---------------- roofline of the dominant kernel
     R = int(layer.outputs["offsets"][-1].item())
-    names = ["router", "scatter", "gemm1", "gemm2", "combine"]  # router includes the fused dispatch scan
+    # router includes the fused dispatch scan; two GEMMs per shared expert before the combine
+    names = ["router", "scatter", "gemm1", "gemm2"] + \
+        [f"shared{i}_gemm{j}" for i in range(wl.n_shared) for j in (1, 2)] + ["combine"]
     assert len(names) == nl, (names, nl)
     mean_stage = stage_ms.mean(axis=0)
     pk, pk_src = peaks()
@@ -286,8 +297,11 @@ def run_native(a):
         "scatter": ("hbm", 2 * R * wl.d * bpe + wl.T * wl.k * 4 * 3),
         "gemm1": ("tensor", gemm1_flops),
         "gemm2": ("tensor", gemm2_flops),
-        "combine": ("hbm", R * wl.d * bpe + wl.T * wl.d * bpe + wl.T * wl.k * 8),
+        "combine": ("hbm", R * wl.d * bpe + (1 + wl.n_shared) * wl.T * wl.d * bpe + wl.T * wl.k * 8),
     }
+    for i in range(wl.n_shared):
+        algo[f"shared{i}_gemm1"] = ("tensor", (4 if wl.act == "swiglu" else 2) * wl.d * wl.ffn * wl.T)
+        algo[f"shared{i}_gemm2"] = ("tensor", 2 * wl.d * wl.ffn * wl.T)
     dom = int(np.argmax(mean_stage))
     dname = names[dom]
     bound, work = algo[dname]
@@ -344,7 +358,7 @@ def run_native(a):
     e2e_ms = e_start.elapsed_time(e_end)
     pipe.check()
     pipe.close()
-    ref_out = layer.forward(x)["out"].cpu()
+    ref_out = layer.forward(x)["out"].cpu()  # the host-buffer paths take no padding mask
     assert torch.equal(outs_host[(a.steps - 1) % depth], ref_out), "pipelined output differs from the forward"
 
     # (b) one synchronous-style call per step (moe_forward_hostio: copy in,

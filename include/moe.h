@@ -121,6 +121,8 @@ typedef struct {
     int32_t router_kernel;     /* moe_router_kernel_t (0: library's choice) */
     int32_t gemm_kernel;       /* moe_gemm_kernel_t (0: library's choice) */
     int32_t dispatch;          /* moe_dispatch_mode_t (0: library's choice) */
+    int32_t n_shared;          /* shared experts, 0..8 (LLaMA4-MoE §5.2; see moe_forward) */
+    int32_t reserved;          /* must be 0 */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */
@@ -132,6 +134,12 @@ typedef struct {
     const void* w_down_or_w2;        /* [E, ffn, d]  SwiGLU W_down | GELU W2 */
     const void* b1;                  /* [E, ffn] GELU only, else NULL */
     const void* b2;                  /* [E, d]   GELU only, else NULL */
+    /* shared experts (n_shared > 0), same form and layout per expert as the routed ones */
+    const void* shared_gate_or_w1;   /* [S, d, ffn] */
+    const void* shared_up;           /* [S, d, ffn] SwiGLU only, else NULL */
+    const void* shared_down_or_w2;   /* [S, ffn, d] */
+    const void* shared_b1;           /* [S, ffn] GELU only, else NULL */
+    const void* shared_b2;           /* [S, d]   GELU only, else NULL */
 } moe_weights_t;
 
 /* Outputs of moe_forward (device).  R_max = moe_max_rows(). */
@@ -176,16 +184,20 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
  *   logits_in [T,E] float32 or NULL: when given, these logits (bias already
  *     included) replace x . W_r + bias -- used to feed both this library and a
  *     reference identical logits.
+ *   token_mask [T] uint8 or NULL: tokens with 0 are padding (LLaMA4-MoE §4.1
+ *     keeps them out of expert selection): their topk_idx is -1 and topk_w 0.
  *   topk_idx [T,k] int32, topk_w [T,k] float32 (outputs).
- *   logits_out, probs_out [T,E] float32 or NULL (optional outputs).
+ *   logits_out, probs_out [T,E] float32 or NULL (optional outputs; written for
+ *     every token, padding included).
  * Top-k compares fp32 logits, lower id first on ties.  Needs a workspace. */
 moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router,
-                             const float* logit_bias, const float* logits_in,
+                             const float* logit_bias, const float* logits_in, const uint8_t* token_mask,
                              int32_t* topk_idx, float* topk_w, float* logits_out, float* probs_out,
                              void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Capacity-bounded dispatch (MoE-basics §2.4; LLaMA4-MoE §2.4).
- *   topk_idx [T,k] int32 in [0,E).  Outputs: counts [E], offsets [E+1],
+ *   topk_idx [T,k] int32 in [0,E), or -1 (selects nothing: padding).
+ *   Outputs: counts [E], offsets [E+1],
  *   slot [T,k], src_assign [R_max] (first offsets[E] entries), and
  *   x_perm [R_max, d] whose row s is x[src_assign[s] / k].
  * Assignment (t,j) has rank = number of earlier assignments (token-major
@@ -235,11 +247,18 @@ moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const
                            float* f, float* p, float* l_aux, cudaStream_t stream);
 
 /* The whole layer forward: router, top-k, dispatch, expert FFNs, combine and
- * aux statistics, five kernel launches on `stream`.  `logits_in` as in
- * moe_router_topk (NULL in normal use). */
+ * aux statistics on `stream` (moe_forward_launch_count launches).
+ *   logits_in as in moe_router_topk (NULL in normal use).
+ *   token_mask [T] uint8 or NULL: padding tokens (0) select no expert, get no
+ *     routed output and are left out of f and p, which divide by the number
+ *     of real tokens; the capacity stays that of the whole batch.
+ *   n_shared > 0: the shared experts (weights->shared_*) run on every token,
+ *     padding included, and out[t] = sum_j w[t,j] y(t,j) + sum_s y_s(t),
+ *     accumulated in fp32 (routed terms first, then shared experts in order)
+ *     and rounded once. */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
-                         const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
-                         cudaStream_t stream);
+                         const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs, void* ws,
+                         size_t ws_bytes, cudaStream_t stream);
 
 /* ---- Data-parallel sharding of one logical batch ----------------------
  * One batch of T_global tokens split in contiguous slices over `world` ranks
@@ -283,8 +302,8 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
  * attributes) and replayed; a replay reads x and the weights as they are at
  * replay time. */
 moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
-                                  const float* logits_in, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
-                                  cudaStream_t stream, cudaEvent_t* stage_events);
+                                  const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs,
+                                  void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t* stage_events);
 
 /* moe_forward with the token activations in HOST memory: copies x_host
  * (HOST, [T,d], pinned for asynchronous copies) to x_dev (device, [T,d]),

@@ -42,12 +42,14 @@ class MoEConfigC(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("ffn", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("router_kernel", ctypes.c_int32),
-                ("gemm_kernel", ctypes.c_int32), ("dispatch", ctypes.c_int32)]
+                ("gemm_kernel", ctypes.c_int32), ("dispatch", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class MoEWeightsC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("w_router", "router_logit_bias", "w_gate_or_w1", "w_up", "w_down_or_w2", "b1", "b2")]
+                ("w_router", "router_logit_bias", "w_gate_or_w1", "w_up", "w_down_or_w2", "b1", "b2",
+                 "shared_gate_or_w1", "shared_up", "shared_down_or_w2", "shared_b1", "shared_b2")]
 
 
 class MoEOutputsC(ctypes.Structure):
@@ -76,15 +78,15 @@ def lib() -> ctypes.CDLL:
     L.moe_max_rows.argtypes = [_CFG, ctypes.POINTER(ctypes.c_int64)]
     L.moe_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
     L.moe_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
-    L.moe_router_topk.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.moe_router_topk.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     L.moe_dispatch.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     L.moe_expert_ffn.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, _P, _P, ctypes.c_size_t, _P]
     L.moe_combine.argtypes = [_CFG, _P, _P, _P, _P, _P]
     L.moe_aux_stats.argtypes = [_CFG, _P, _P, _P, _P, _P, _P]
-    L.moe_forward.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P,
+    L.moe_forward.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, _P, ctypes.POINTER(MoEOutputsC), _P,
                               ctypes.c_size_t, _P]
-    L.moe_forward_profiled.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P,
-                                       ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_forward_profiled.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, _P, ctypes.POINTER(MoEOutputsC),
+                                       _P, ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_void_p)]
     L.moe_forward_hostio.argtypes = [_CFG, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P, _P,
                                      _P, ctypes.c_size_t, _P]
     L.moe_check_device_status.argtypes = [_P, ctypes.c_size_t, _P, ctypes.POINTER(ctypes.c_uint32)]
@@ -125,13 +127,14 @@ class MoEConfig:
     router_kernel: str = "auto"  # "auto" | "warp_mma" | "tcgen05"
     gemm_kernel: str = "auto"    # "auto" | "one_cta" | "cta_pair"
     dispatch: str = "auto"       # "auto" | "copy" | "gather"
+    n_shared: int = 0            # shared experts, applied to every token with weight 1
 
     def c(self) -> MoEConfigC:
         return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
                           MOE_DT_BF16 if self.dtype == "bf16" else MOE_DT_F32,
                           MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
                           float(self.capacity_factor), float(self.aux_alpha), ROUTER_KERNELS[self.router_kernel],
-                          GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch])
+                          GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch], int(self.n_shared), 0)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -141,7 +144,7 @@ class MoEConfig:
     def of(wl, router_kernel: str = "auto", gemm_kernel: str = "auto", dispatch: str = "auto") -> "MoEConfig":
         """From a workload description (anything with the same field names)."""
         return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha,
-                         router_kernel, gemm_kernel, dispatch)
+                         router_kernel, gemm_kernel, dispatch, getattr(wl, "n_shared", 0))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -200,10 +203,10 @@ def moe_workspace_init(ws: Workspace, stream=None) -> None:
 
 
 def moe_router_topk(cfg: MoEConfig, x, w_router, logit_bias, logits_in, topk_idx, topk_w, logits_out, probs_out,
-                    ws: Workspace, stream=None) -> None:
+                    ws: Workspace, stream=None, token_mask=None) -> None:
     _check(lib().moe_router_topk(ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(logit_bias), _ptr(logits_in),
-                                 _ptr(topk_idx), _ptr(topk_w), _ptr(logits_out), _ptr(probs_out), ws.ptr, ws.nbytes,
-                                 _stream(stream)), "moe_router_topk")
+                                 _ptr(token_mask), _ptr(topk_idx), _ptr(topk_w), _ptr(logits_out), _ptr(probs_out),
+                                 ws.ptr, ws.nbytes, _stream(stream)), "moe_router_topk")
 
 
 def moe_dispatch(cfg: MoEConfig, x, topk_idx, counts, offsets, slot, src_assign, x_perm, ws: Workspace,
@@ -213,9 +216,14 @@ def moe_dispatch(cfg: MoEConfig, x, topk_idx, counts, offsets, slot, src_assign,
 
 
 def _weights_c(w: dict) -> MoEWeightsC:
+    """Weights by name: w_router, router_bias, w_gate/w_up/w_down (SwiGLU) or
+    w1/b1/w2/b2 (GELU), and the shared experts' shared_gate/shared_up/
+    shared_down or shared_w1/shared_b1/shared_w2/shared_b2."""
     g = lambda n: _ptr(w.get(n))  # noqa: E731
     return MoEWeightsC(g("w_router"), g("router_bias"), g("w_gate") if "w_gate" in w else g("w1"), g("w_up"),
-                       g("w_down") if "w_down" in w else g("w2"), g("b1"), g("b2"))
+                       g("w_down") if "w_down" in w else g("w2"), g("b1"), g("b2"),
+                       g("shared_gate") if "shared_gate" in w else g("shared_w1"), g("shared_up"),
+                       g("shared_down") if "shared_down" in w else g("shared_w2"), g("shared_b1"), g("shared_b2"))
 
 
 def moe_expert_ffn(cfg: MoEConfig, weights: dict, x_perm, offsets, y_perm, ws: Workspace, stream=None) -> None:
@@ -263,22 +271,23 @@ def allocate_outputs(cfg: MoEConfig, device="cuda", with_logits: bool = False, w
     return o
 
 
-def moe_forward(cfg: MoEConfig, weights: dict, x, outputs: dict, ws: Workspace, logits_in=None, stream=None) -> None:
+def moe_forward(cfg: MoEConfig, weights: dict, x, outputs: dict, ws: Workspace, logits_in=None, stream=None,
+                token_mask=None) -> None:
     wc = _weights_c(weights)
     oc = _outputs_c(outputs)
-    _check(lib().moe_forward(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x), _ptr(logits_in), ctypes.byref(oc),
-                             ws.ptr, ws.nbytes, _stream(stream)), "moe_forward")
+    _check(lib().moe_forward(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x), _ptr(logits_in), _ptr(token_mask),
+                             ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)), "moe_forward")
 
 
 def moe_forward_profiled(cfg: MoEConfig, weights: dict, x, outputs: dict, ws: Workspace, events: list,
-                         logits_in=None, stream=None) -> None:
+                         logits_in=None, stream=None, token_mask=None) -> None:
     """moe_forward recording torch.cuda.Event objects `events` (n+1 of them,
     n = moe_forward_launch_count) around each kernel launch on `stream`."""
     wc = _weights_c(weights)
     oc = _outputs_c(outputs)
     arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
     _check(lib().moe_forward_profiled(ctypes.byref(cfg.c()), ctypes.byref(wc), _ptr(x), _ptr(logits_in),
-                                      ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream), arr),
+                                      _ptr(token_mask), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream), arr),
            "moe_forward_profiled")
 
 
@@ -321,22 +330,24 @@ class MoELayer:
         self.outputs = allocate_outputs(cfg, device, with_logits, with_probs)
         self.ws = Workspace(cfg, device)
 
-    def forward(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None, stream=None) -> dict:
-        moe_forward(self.cfg, self.weights, x, self.outputs, self.ws, logits_in, stream)
+    def forward(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None, stream=None,
+                token_mask: Optional[torch.Tensor] = None) -> dict:
+        moe_forward(self.cfg, self.weights, x, self.outputs, self.ws, logits_in, stream, token_mask)
         return self.outputs
 
-    def capture(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
+    def capture(self, x: torch.Tensor, logits_in: Optional[torch.Tensor] = None,
+                token_mask: Optional[torch.Tensor] = None) -> "torch.cuda.CUDAGraph":
         """Records one forward on the fixed buffers `x` / `logits_in` into a CUDA
         graph (five kernel launches, no host work when replayed).  A replay
         reads `x` as it is at that time; results land in `self.outputs`."""
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
-            self.forward(x, logits_in)  # uncaptured first call: kernel attributes, cached launch shapes
+            self.forward(x, logits_in, token_mask=token_mask)  # uncaptured first call: kernel attributes
         torch.cuda.current_stream().wait_stream(side)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self.forward(x, logits_in)
+            self.forward(x, logits_in, token_mask=token_mask)
         self.graph = g
         return g
 

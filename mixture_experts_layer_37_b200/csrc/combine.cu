@@ -4,8 +4,10 @@
 // Combine: out[t] = sum_j w[t,j] * expert_j(x[t]) ("Hand-building a
 // LLaMA4-MoE" (dpshk.com/news/5809432) §2.4; "MoE: gating, experts, load
 // balancing, capacity factor" (dpshk.com/news/6005940) §3.1), over the kept
-// assignments only, fp32 accumulation in ascending j.  One warp per token,
-// 16-byte vector loads of the expert rows, no atomics.
+// assignments only, fp32 accumulation in ascending j, then plus each shared
+// expert's output (LLaMA4-MoE §5.2: fixed experts in every token's
+// computation), rounded once.  One warp per token, 16-byte vector loads of
+// the expert rows, no atomics.
 //
 // Statistics: f_e = n_e / (T*k), p_e = mean_t softmax[t,e],
 // L_aux = alpha * E * sum_e f_e p_e (MoE-basics §2.3 and §3.1).
@@ -78,6 +80,32 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
                             acc[u][2] = fmaf(w, __uint_as_float(yv.z), acc[u][2]);
                             acc[u][3] = fmaf(w, __uint_as_float(yv.w), acc[u][3]);
                         }
+                    }
+                }
+            }
+            // shared experts: every token, weight 1, after the routed terms, in order
+            for (int sh = 0; sh < a.n_shared; ++sh) {
+                const uint4* YS = reinterpret_cast<const uint4*>(a.y_shared) + ((int64_t)sh * a.T + t) * nvec;
+                uint4 ysv[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (v0 + 32 * u < nvec) ysv[u] = YS[v0 + 32 * u];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (v0 + 32 * u >= nvec) continue;
+                    const uint4 yv = ysv[u];
+                    if constexpr (BF16) {
+                        const uint32_t ys[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            acc[u][2 * q] += bf16_lo(ys[q]);
+                            acc[u][2 * q + 1] += bf16_hi(ys[q]);
+                        }
+                    } else {
+                        acc[u][0] += __uint_as_float(yv.x);
+                        acc[u][1] += __uint_as_float(yv.y);
+                        acc[u][2] += __uint_as_float(yv.z);
+                        acc[u][3] += __uint_as_float(yv.w);
                     }
                 }
             }

@@ -36,8 +36,8 @@ enum WaitSite : uint32_t {
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 struct DevStatus {
-    uint32_t* word;       // [0] error bits, [1] first site, [2] never-set flag
-    uint64_t timeout_ns;  // limit of every bounded wait
+    uint32_t* word = nullptr;  // [0] error bits, [1] first site, [2] never-set flag
+    uint64_t timeout_ns = 0;   // limit of every bounded wait
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

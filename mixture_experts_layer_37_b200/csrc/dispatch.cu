@@ -163,6 +163,10 @@ __global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
         }
         a.offsets[a.E] = off;
         a.l_aux[0] = (float)((double)a.alpha * a.E * l);
+        if (a.shared_off != nullptr) {
+            a.shared_off[0] = 0;
+            a.shared_off[1] = (int32_t)a.T_local;
+        }
     }
 }
 

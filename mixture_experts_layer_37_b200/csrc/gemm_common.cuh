@@ -39,18 +39,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 }
 
 struct GemmParams {
-    const int32_t* offsets;      // [E+1] kept-row offsets per expert
-    __nv_bfloat16* out;          // [rows_cap, N]
-    const __nv_bfloat16* bias;   // [E, N] or null
-    int E, K, N;
-    int bn_out;                  // output columns per tile: 128 (SwiGLU) or 256
-    int n_tiles;
+    const int32_t* offsets = nullptr;     // [E+1] kept-row offsets per expert
+    __nv_bfloat16* out = nullptr;         // [rows_cap, N]
+    const __nv_bfloat16* bias = nullptr;  // [E, N] or null
+    int E = 0, K = 0, N = 0;
+    int bn_out = 0;                       // output columns per tile: 128 (SwiGLU) or 256
+    int n_tiles = 0;
     DevStatus st;
     // A rows gathered from the token activations instead of a sorted copy:
     // row s of the expert-sorted order is token src_assign[s] / k of gx
-    const __nv_bfloat16* gx;     // [T, K] or null (A read through its tensor map)
-    const int32_t* src_assign;   // [R]
-    int k;
+    const __nv_bfloat16* gx = nullptr;    // [T, K] or null (A read through its tensor map)
+    const int32_t* src_assign = nullptr;  // [R]
+    int k = 0;
 };
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }

@@ -11,41 +11,45 @@
 namespace moe {
 
 struct ScanArgs {
-    const int32_t* hist;   // [E, nchunk] per-chunk expert histogram
-    const double* psum;    // [E, nchunk] per-chunk probability sums, or null (no aux stats)
-    int32_t* chunk_base;   // [E, nchunk] out: assignments to e in earlier chunks
-    int32_t* counts;       // [E] out
-    int32_t* offsets;      // [E+1] out
-    float* f;              // [E] out or null
-    float* p;              // [E] out or null
-    float* l_aux;          // [1] out or null
-    double* psum_total;    // [E] out or null: sum over this batch's tokens of p[t,e] (not divided)
-    int64_t T;
-    int nchunk, E, k, cap;
-    float alpha;
+    const int32_t* hist = nullptr;   // [E, nchunk] per-chunk expert histogram
+    const double* psum = nullptr;    // [E, nchunk] per-chunk probability sums, or null (no aux stats)
+    int32_t* chunk_base = nullptr;   // [E, nchunk] out: assignments to e in earlier chunks
+    int32_t* counts = nullptr;       // [E] out
+    int32_t* offsets = nullptr;      // [E+1] out
+    float* f = nullptr;              // [E] out or null
+    float* p = nullptr;              // [E] out or null
+    float* l_aux = nullptr;          // [1] out or null
+    double* psum_total = nullptr;    // [E] out or null: sum over this batch's tokens of p[t,e] (not divided)
+    const int32_t* nreal = nullptr;  // [nchunk] real (unmasked) tokens per chunk, or null: every token is real
+    int32_t* shared_off = nullptr;   // [2] out or null: {0, T}, the row offsets of the shared experts' GEMMs
+    int64_t T = 0;
+    int nchunk = 0, E = 0, k = 0, cap = 0;
+    float alpha = 0;
 };
 
 struct RouterArgs {
-    const void* x;           // [T, d] act dtype
-    const void* w_router;    // [d, E] act dtype
-    const float* bias;       // [E] or null
-    const float* logits_in;  // [T, E] or null
-    int32_t* topk_idx;       // [T, k]
-    float* topk_w;           // [T, k]
-    float* logits_out;       // [T, E] or null
-    float* probs_out;        // [T, E] or null
-    int32_t* hist;           // [E, nchunk] per-chunk expert histogram
-    double* psum;            // [E, nchunk] per-chunk sum of probabilities
-    int64_t T;
-    int d, E, k, nchunk;
-    int tpc;                 // tokens per CTA (set by the launcher; multiple of the chunk)
+    const void* x = nullptr;           // [T, d] act dtype
+    const void* w_router = nullptr;    // [d, E] act dtype
+    const float* bias = nullptr;       // [E] or null
+    const float* logits_in = nullptr;  // [T, E] or null
+    int32_t* topk_idx = nullptr;       // [T, k]
+    float* topk_w = nullptr;           // [T, k]
+    float* logits_out = nullptr;       // [T, E] or null
+    float* probs_out = nullptr;        // [T, E] or null
+    int32_t* hist = nullptr;           // [E, nchunk] per-chunk expert histogram
+    double* psum = nullptr;            // [E, nchunk] per-chunk sum of probabilities
+    const uint8_t* mask = nullptr;     // [T] 0 = padding token (selects nothing, not in the sums), or null
+    int32_t* nreal = nullptr;          // [nchunk] out: real tokens per chunk (written when mask != null)
+    int64_t T = 0;
+    int d = 0, E = 0, k = 0, nchunk = 0;
+    int tpc = 0;                 // tokens per CTA (set by the launcher; multiple of the chunk)
     // when fuse_scan != 0: the last CTA to finish (counted on `counter`) runs
     // the dispatch scan and the aux statistics described by `scan`
-    int fuse_scan;
-    unsigned int* counter;
+    int fuse_scan = 0;
+    unsigned int* counter = nullptr;
     ScanArgs scan;
     DevStatus st;            // status word and wait limit (tensor-core router)
-    int kernel;              // moe_router_kernel_t
+    int kernel = 0;              // moe_router_kernel_t
 };
 cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
 // Tensor-core router (TMA + tcgen05 + TMEM): bf16, E % 8 == 0, no logits feed.
@@ -56,17 +60,17 @@ cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t
 cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s);
 
 struct ScatterArgs {
-    const int32_t* topk_idx;    // [T, k]
-    const int32_t* chunk_base;  // [E, nchunk]
-    const int32_t* offsets;     // [E+1]
-    int32_t* slot;              // [T, k]
-    int32_t* src_assign;        // [R_max]
-    const void* x;              // [T, d]
-    void* x_perm;               // [R_max, d], or null: no row copies (slot / src_assign only)
-    const int32_t* cap_e;       // [E] per-expert capacity left for this batch, or null (use cap)
-    int64_t T;
-    int E, k, cap, nchunk;
-    int row_bytes;              // d * element size (multiple of 16)
+    const int32_t* topk_idx = nullptr;    // [T, k]
+    const int32_t* chunk_base = nullptr;  // [E, nchunk]
+    const int32_t* offsets = nullptr;     // [E+1]
+    int32_t* slot = nullptr;              // [T, k]
+    int32_t* src_assign = nullptr;        // [R_max]
+    const void* x = nullptr;              // [T, d]
+    void* x_perm = nullptr;               // [R_max, d], or null: no row copies (slot / src_assign only)
+    const int32_t* cap_e = nullptr;       // [E] per-expert capacity left for this batch, or null (use cap)
+    int64_t T = 0;
+    int E = 0, k = 0, cap = 0, nchunk = 0;
+    int row_bytes = 0;              // d * element size (multiple of 16)
 };
 cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
 
@@ -74,27 +78,31 @@ cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
 // probability sums ([world, E], gathered in rank order) compute this rank's
 // per-expert capacity left, kept offsets, and the global counts / f / p / L_aux.
 struct DpPrepareArgs {
-    const int32_t* all_counts;  // [world, E]
-    const double* all_psum;     // [world, E]
-    int world, rank, E, k, cap;
-    int64_t T_global;
-    float alpha;
-    int32_t* cap_e;             // [E] out
-    int32_t* offsets;           // [E+1] out (this rank's kept rows)
-    int32_t* counts;            // [E] out (global)
-    float* f;                   // [E] out
-    float* p;                   // [E] out
-    float* l_aux;               // [1] out
+    const int32_t* all_counts = nullptr;  // [world, E]
+    const double* all_psum = nullptr;     // [world, E]
+    int world = 0, rank = 0, E = 0, k = 0, cap = 0;
+    int64_t T_global = 0;
+    float alpha = 0;
+    int32_t* cap_e = nullptr;             // [E] out
+    int32_t* offsets = nullptr;           // [E+1] out (this rank's kept rows)
+    int32_t* counts = nullptr;            // [E] out (global)
+    float* f = nullptr;                   // [E] out
+    float* p = nullptr;                   // [E] out
+    float* l_aux = nullptr;               // [1] out
+    int32_t* shared_off = nullptr;        // [2] out or null: {0, T_local}, the shared experts' row offsets
+    int64_t T_local = 0;
 };
 cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s);
 
 struct CombineArgs {
-    const void* y_perm;    // [R_max, d]
-    const int32_t* slot;   // [T, k]
-    const float* topk_w;   // [T, k]
-    void* out;             // [T, d]
-    int64_t T;
-    int d, k;
+    const void* y_perm = nullptr;    // [R_max, d]
+    const int32_t* slot = nullptr;   // [T, k]
+    const float* topk_w = nullptr;   // [T, k]
+    void* out = nullptr;             // [T, d]
+    const void* y_shared = nullptr;  // [n_shared, T, d] shared experts' outputs, added with weight 1, or null
+    int n_shared = 0;
+    int64_t T = 0;
+    int d = 0, k = 0;
 };
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_aux_from_probs(const int32_t* counts, const float* probs, float* f, float* p, float* l_aux,
@@ -102,26 +110,26 @@ cudaError_t launch_aux_from_probs(const int32_t* counts, const float* probs, flo
 
 // Expert FFN (grouped GEMMs over the expert-sorted rows).
 struct FfnArgs {
-    int act;                 // 0 swiglu, 1 gelu+bias
-    int E, d, ffn;
-    int64_t rows_cap;        // R_max (rows allocated in x_perm / h / y_perm)
-    const int32_t* offsets;  // [E+1]
-    const void* x_perm;      // [rows_cap, d]
-    void* h;                 // [rows_cap, ffn] (workspace)
-    void* y_perm;            // [rows_cap, d]
-    const void* w1;          // [E, d, ffn] (gate or W1)
-    const void* w_up;        // [E, d, ffn] or null
-    const void* w2;          // [E, ffn, d]
-    const void* b1;          // [E, ffn] or null
-    const void* b2;          // [E, d] or null
+    int act = 0;                 // 0 swiglu, 1 gelu+bias
+    int E = 0, d = 0, ffn = 0;
+    int64_t rows_cap = 0;        // R_max (rows allocated in x_perm / h / y_perm)
+    const int32_t* offsets = nullptr;  // [E+1]
+    const void* x_perm = nullptr;      // [rows_cap, d]
+    void* h = nullptr;                 // [rows_cap, ffn] (workspace)
+    void* y_perm = nullptr;            // [rows_cap, d]
+    const void* w1 = nullptr;          // [E, d, ffn] (gate or W1)
+    const void* w_up = nullptr;        // [E, d, ffn] or null
+    const void* w2 = nullptr;          // [E, ffn, d]
+    const void* b1 = nullptr;          // [E, ffn] or null
+    const void* b2 = nullptr;          // [E, d] or null
     DevStatus st;
-    cudaEvent_t between;     // recorded between the two GEMM launches, or null
-    int gemm_kernel;         // moe_gemm_kernel_t
+    cudaEvent_t between = nullptr;  // recorded between the two GEMM launches, or null
+    int gemm_kernel = 0;         // moe_gemm_kernel_t
     // when gather_x != null the first GEMM reads its rows straight from the
     // tokens (row s = token src_assign[s] / k) and x_perm is not used
-    const void* gather_x;    // [T, d] or null
-    const int32_t* src_assign;
-    int k;
+    const void* gather_x = nullptr;    // [T, d] or null
+    const int32_t* src_assign = nullptr;
+    int k = 0;
 };
 // bf16: tcgen05 grouped GEMMs (two launches).  Returns cudaErrorInvalidValue
 // when a tensor map cannot be encoded.

@@ -35,6 +35,7 @@ using namespace moe;
 uint32_t g_timeout_ms = 2000;
 
 constexpr size_t kStatusBytes = 1024;
+constexpr int kMaxShared = 8;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -48,8 +49,9 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
         c->router_kernel > MOE_ROUTER_TCGEN05 || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
-        c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER)
+        c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER || c->n_shared < 0 || c->reserved != 0)
         return MOE_ERR_INVALID_ARG;
+    if (c->n_shared > kMaxShared) return MOE_ERR_UNSUPPORTED;
     if (c->router_kernel == MOE_ROUTER_TCGEN05 &&
         (c->dtype != MOE_DT_BF16 || c->E % 8 != 0 || c->d % 64 != 0))
         return MOE_ERR_UNSUPPORTED;
@@ -86,7 +88,7 @@ int64_t max_rows(const moe_config_t* c) {
 struct Plan {
     int nchunk;
     int64_t rows;
-    size_t hist, psum, base, cap_e, xperm, h, yperm, total;
+    size_t hist, psum, base, cap_e, nreal, shared_off, xperm, h, yperm, hs, ys, total;
 };
 
 Plan plan_rows(const moe_config_t* c, int64_t rows) {
@@ -104,12 +106,21 @@ Plan plan_rows(const moe_config_t* c, int64_t rows) {
     off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
     p.cap_e = off;
     off = align_up(off + E * 4, 1024);
+    p.nreal = off;
+    off = align_up(off + (size_t)p.nchunk * 4, 1024);
+    p.shared_off = off;
+    off = align_up(off + 2 * 4, 1024);
     p.xperm = off;
     off = align_up(off + (size_t)p.rows * c->d * s, 1024);
     p.h = off;
     off = align_up(off + (size_t)p.rows * c->ffn * s, 1024);
     p.yperm = off;
     off = align_up(off + (size_t)p.rows * c->d * s, 1024);
+    // shared experts: one [T, ffn] intermediate reused in turn, and each one's [T, d] output
+    p.hs = off;
+    off = align_up(off + (c->n_shared > 0 ? (size_t)c->T * c->ffn * s : 0), 1024);
+    p.ys = off;
+    off = align_up(off + (size_t)c->n_shared * c->T * c->d * s, 1024);
     p.total = off;
     return p;
 }
@@ -172,6 +183,17 @@ moe_status_t check_weights(const moe_config_t* c, const moe_weights_t* w, bool n
             if (w->b1 == nullptr || w->b2 == nullptr || !aligned16(w->b1) || !aligned16(w->b2))
                 return MOE_ERR_INVALID_ARG;
         }
+        if (c->n_shared > 0) {
+            if (w->shared_gate_or_w1 == nullptr || w->shared_down_or_w2 == nullptr ||
+                !aligned16(w->shared_gate_or_w1) || !aligned16(w->shared_down_or_w2))
+                return MOE_ERR_INVALID_ARG;
+            if (c->act == MOE_ACT_SWIGLU) {
+                if (w->shared_up == nullptr || !aligned16(w->shared_up)) return MOE_ERR_INVALID_ARG;
+            } else if (w->shared_b1 == nullptr || w->shared_b2 == nullptr || !aligned16(w->shared_b1) ||
+                       !aligned16(w->shared_b2)) {
+                return MOE_ERR_INVALID_ARG;
+            }
+        }
     }
     return MOE_OK;
 }
@@ -188,6 +210,8 @@ ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, flo
     sa.p = p;
     sa.l_aux = l_aux;
     sa.psum_total = nullptr;
+    sa.nreal = nullptr;
+    sa.shared_off = c->n_shared > 0 ? reinterpret_cast<int32_t*>(at(ws, pl.shared_off)) : nullptr;
     sa.T = c->T;
     sa.nchunk = pl.nchunk;
     sa.E = c->E;
@@ -199,8 +223,8 @@ ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, flo
 
 // Router; with `fused` set, its last CTA also runs the scan described by `sa`.
 moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_router, const float* bias,
-                        const float* logits_in, int32_t* idx, float* w, float* logits_out, float* probs_out,
-                        void* ws, const Plan& pl, cudaStream_t s, const ScanArgs* fused = nullptr) {
+                        const float* logits_in, const uint8_t* mask, int32_t* idx, float* w, float* logits_out,
+                        float* probs_out, void* ws, const Plan& pl, cudaStream_t s, const ScanArgs* fused = nullptr) {
     RouterArgs a;
     a.x = x;
     a.w_router = w_router;
@@ -212,6 +236,8 @@ moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_rout
     a.probs_out = probs_out;
     a.hist = reinterpret_cast<int32_t*>(at(ws, pl.hist));
     a.psum = reinterpret_cast<double*>(at(ws, pl.psum));
+    a.mask = mask;
+    a.nreal = reinterpret_cast<int32_t*>(at(ws, pl.nreal));
     a.T = c->T;
     a.d = c->d;
     a.E = c->E;
@@ -219,7 +245,10 @@ moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_rout
     a.nchunk = pl.nchunk;
     a.fuse_scan = fused != nullptr ? 1 : 0;
     a.counter = static_cast<unsigned int*>(ws) + kStatusCounterWord;
-    if (fused != nullptr) a.scan = *fused;
+    if (fused != nullptr) {
+        a.scan = *fused;
+        if (mask != nullptr) a.scan.nreal = a.nreal;  // statistics over the real tokens
+    }
     a.st = status_of(ws);
     a.kernel = c->router_kernel;
     return from_cuda(launch_router(a, c->dtype == MOE_DT_BF16, s));
@@ -278,16 +307,55 @@ moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* 
 }
 
 moe_status_t run_combine(const moe_config_t* c, const void* y_perm, const int32_t* slot, const float* w, void* out,
-                         cudaStream_t s) {
+                         cudaStream_t s, const void* y_shared = nullptr) {
     CombineArgs a;
     a.y_perm = y_perm;
     a.slot = slot;
     a.topk_w = w;
     a.out = out;
+    a.y_shared = y_shared;
+    a.n_shared = y_shared != nullptr ? c->n_shared : 0;
     a.T = c->T;
     a.d = c->d;
     a.k = c->k;
     return from_cuda(launch_combine(a, c->dtype == MOE_DT_BF16, s));
+}
+
+// The shared experts (LLaMA4-MoE §5.2): each one's two GEMMs over all T token
+// rows (one group of T rows, offsets {0, T} written by the scan), its output in
+// ys[s].  `mark` records the stage events of moe_forward_profiled.
+template <class Mark>
+moe_status_t run_shared(const moe_config_t* c, const moe_weights_t* w, const void* x, void* ws, const Plan& pl,
+                        cudaStream_t s, Mark&& mark, cudaEvent_t* ev, int* n) {
+    const size_t es = elem_size(c);
+    const size_t wsz = (size_t)c->d * c->ffn * es;
+    for (int i = 0; i < c->n_shared; ++i) {
+        FfnArgs f;
+        f.act = c->act;
+        f.E = 1;
+        f.d = c->d;
+        f.ffn = c->ffn;
+        f.rows_cap = c->T;
+        f.offsets = reinterpret_cast<const int32_t*>(at(ws, pl.shared_off));
+        f.x_perm = x;
+        f.h = at(ws, pl.hs);
+        f.y_perm = at(ws, pl.ys + (size_t)i * c->T * c->d * es);
+        f.w1 = static_cast<const uint8_t*>(w->shared_gate_or_w1) + i * wsz;
+        f.w_up = w->shared_up != nullptr ? static_cast<const uint8_t*>(w->shared_up) + i * wsz : nullptr;
+        f.w2 = static_cast<const uint8_t*>(w->shared_down_or_w2) + i * wsz;
+        f.b1 = w->shared_b1 != nullptr ? static_cast<const uint8_t*>(w->shared_b1) + (size_t)i * c->ffn * es : nullptr;
+        f.b2 = w->shared_b2 != nullptr ? static_cast<const uint8_t*>(w->shared_b2) + (size_t)i * c->d * es : nullptr;
+        f.st = status_of(ws);
+        f.between = ev != nullptr ? ev[(*n)++] : nullptr;
+        f.gemm_kernel = c->gemm_kernel;
+        f.gather_x = nullptr;
+        f.src_assign = nullptr;
+        f.k = 1;
+        const cudaError_t e = c->dtype == MOE_DT_BF16 ? launch_ffn_bf16_sm100(f, s) : launch_ffn_f32(f, s);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (!mark()) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
 }
 
 }  // namespace
@@ -336,8 +404,8 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) 
 }
 
 moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void* w_router, const float* logit_bias,
-                             const float* logits_in, int32_t* topk_idx, float* topk_w, float* logits_out,
-                             float* probs_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                             const float* logits_in, const uint8_t* token_mask, int32_t* topk_idx, float* topk_w,
+                             float* logits_out, float* probs_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
     if (topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
@@ -347,7 +415,8 @@ moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void*
     Plan pl;
     if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
     if (cfg->T == 0) return MOE_OK;
-    return run_router(cfg, x, w_router, logit_bias, logits_in, topk_idx, topk_w, logits_out, probs_out, ws, pl, stream);
+    return run_router(cfg, x, w_router, logit_bias, logits_in, token_mask, topk_idx, topk_w, logits_out, probs_out, ws,
+                      pl, stream);
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
@@ -403,8 +472,8 @@ moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const
 }
 
 static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
-                                 const float* logits_in, moe_outputs_t* o, void* ws, size_t ws_bytes,
-                                 cudaStream_t stream, cudaEvent_t* ev) {
+                                 const float* logits_in, const uint8_t* token_mask, moe_outputs_t* o, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream, cudaEvent_t* ev) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
     if ((st = check_weights(cfg, weights, logits_in == nullptr, true)) != MOE_OK) return st;
@@ -429,8 +498,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     void* x_perm = at(ws, pl.xperm);
     void* y_perm = at(ws, pl.yperm);
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
-                    o->logits_out, o->probs_out, ws, pl, stream, &sa);
+    st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, token_mask, o->topk_idx,
+                    o->topk_w, o->logits_out, o->probs_out, ws, pl, stream, &sa);
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
     const bool gather = gathers(cfg);
@@ -442,21 +511,23 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
                  gather ? x : nullptr, o->src_assign);
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
+    if ((st = run_shared(cfg, weights, x, ws, pl, stream, mark, ev, &n)) != MOE_OK) return st;
+    st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
+                     cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
     if (st != MOE_OK) return st;
     return mark() ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, const float* logits_in,
-                         moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    return forward_impl(cfg, weights, x, logits_in, o, ws, ws_bytes, stream, nullptr);
+                         const uint8_t* token_mask, moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    return forward_impl(cfg, weights, x, logits_in, token_mask, o, ws, ws_bytes, stream, nullptr);
 }
 
 moe_status_t moe_forward_profiled(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
-                                  const float* logits_in, moe_outputs_t* o, void* ws, size_t ws_bytes,
-                                  cudaStream_t stream, cudaEvent_t* stage_events) {
+                                  const float* logits_in, const uint8_t* token_mask, moe_outputs_t* o, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream, cudaEvent_t* stage_events) {
     if (stage_events == nullptr) return MOE_ERR_INVALID_ARG;
-    return forward_impl(cfg, weights, x, logits_in, o, ws, ws_bytes, stream, stage_events);
+    return forward_impl(cfg, weights, x, logits_in, token_mask, o, ws, ws_bytes, stream, stage_events);
 }
 
 moe_status_t moe_dp_workspace_size(const moe_config_t* cfg, int64_t T_global, size_t* bytes) {
@@ -494,7 +565,7 @@ moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_w
     sa.cap = 0x7fffffff;        // local totals only; the capacity is applied in moe_dp_finish
     sa.psum_total = local_psum;
     if (cfg->T == 0) return from_cuda(launch_dispatch_scan(sa, stream));
-    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, o->topk_idx, o->topk_w,
+    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, nullptr, o->topk_idx, o->topk_w,
                       o->logits_out, o->probs_out, ws, pl, stream, &sa);
 }
 
@@ -532,6 +603,8 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
     dp.f = o->f;
     dp.p = o->p;
     dp.l_aux = o->l_aux;
+    dp.shared_off = cfg->n_shared > 0 ? reinterpret_cast<int32_t*>(at(ws, pl.shared_off)) : nullptr;
+    dp.T_local = cfg->T;
     if (launch_dp_prepare(dp, stream) != cudaSuccess) return MOE_ERR_CUDA;
     if (cfg->T == 0) return MOE_OK;
     void* x_perm = at(ws, pl.xperm);
@@ -543,7 +616,14 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
     st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, nullptr, gather ? x : nullptr,
                  o->src_assign);
     if (st != MOE_OK) return st;
-    return run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream);
+    if (cfg->n_shared > 0) {
+        // the shared experts' row offsets {0, T} were written by the prepare kernel
+        auto nomark = []() { return true; };
+        int n = 0;
+        if ((st = run_shared(cfg, weights, x, ws, pl, stream, nomark, nullptr, &n)) != MOE_OK) return st;
+    }
+    return run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
+                       cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
 }
 
 moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_host,
@@ -556,7 +636,7 @@ moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* we
     if (cfg->T > 0 && (x_host == nullptr || x_dev == nullptr || out_host == nullptr)) return MOE_ERR_INVALID_ARG;
     if (bytes && cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
         return MOE_ERR_CUDA;
-    st = moe_forward(cfg, weights, x_dev, nullptr, o, ws, ws_bytes, stream);
+    st = moe_forward(cfg, weights, x_dev, nullptr, nullptr, o, ws, ws_bytes, stream);
     if (st != MOE_OK) return st;
     if (bytes && cudaMemcpyAsync(out_host, o->out, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -593,7 +673,7 @@ moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint32_t timeo
 int32_t moe_forward_launch_count(const moe_config_t* cfg) {
     if (check_config(cfg) != MOE_OK) return 0;
     if (cfg->T == 0) return 1;
-    return 5;
+    return 5 + 2 * cfg->n_shared;  // router, scatter, two GEMMs, combine; two GEMMs per shared expert
 }
 
 }  // extern "C"

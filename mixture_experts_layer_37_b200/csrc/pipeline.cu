@@ -166,7 +166,8 @@ moe_status_t moe_pipeline_submit(moe_pipeline_t* p, const void* x_host, void* ou
     cuda_ok(cudaStreamWaitEvent(p->s_comp, p->in_done[s], 0));
     cuda_ok(cudaStreamWaitEvent(p->s_comp, p->out_done[s], 0));
     if (st == MOE_OK)
-        st = moe_forward(&p->cfg, &p->weights, p->x_dev[s], nullptr, &p->outs[s], p->ws, p->ws_bytes, p->s_comp);
+        st = moe_forward(&p->cfg, &p->weights, p->x_dev[s], nullptr, nullptr, &p->outs[s], p->ws, p->ws_bytes,
+                         p->s_comp);
     cuda_ok(cudaEventRecord(p->comp_done[s], p->s_comp));
     // copy out
     cuda_ok(cudaStreamWaitEvent(p->s_out, p->comp_done[s], 0));

@@ -89,6 +89,7 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
     __syncthreads();
     if (tid < ntok) {
         const int64_t t = t0 + tid;
+        const bool real = a.mask == nullptr || a.mask[t] != 0;  // padding selects nothing
         float* row = sL + tid * kLStride;
         float m = -INFINITY;
         for (int e = 0; e < E; ++e) {
@@ -133,10 +134,12 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
         for (int j = 0; j < k; ++j) ps += row[sel_idx[j]];
         int* hrow = sHist + (tid / kChunkTokens) * kMaxExperts;
         for (int j = 0; j < k; ++j) {
-            a.topk_idx[t * k + j] = sel_idx[j];
-            a.topk_w[t * k + j] = row[sel_idx[j]] / ps;
-            atomicAdd(&hrow[sel_idx[j]], 1);
+            a.topk_idx[t * k + j] = real ? sel_idx[j] : -1;
+            a.topk_w[t * k + j] = real ? row[sel_idx[j]] / ps : 0.f;
+            if (real) atomicAdd(&hrow[sel_idx[j]], 1);
         }
+        if (!real)
+            for (int e = 0; e < E; ++e) row[e] = 0.f;  // out of the probability sums
     }
     __syncthreads();
     for (int i = tid; i < nchk * E; i += blockDim.x) {
@@ -147,6 +150,14 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
         a.psum[(int64_t)e * a.nchunk + chunk0 + cl] = acc;
         a.hist[(int64_t)e * a.nchunk + chunk0 + cl] = sHist[cl * kMaxExperts + e];
     }
+    if (a.mask != nullptr)
+        for (int cl = tid; cl < nchk; cl += blockDim.x) {
+            const int64_t c0 = t0 + (int64_t)cl * kChunkTokens;
+            const int64_t c1 = min64(c0 + kChunkTokens, a.T);
+            int n = 0;
+            for (int64_t t = c0; t < c1; ++t) n += a.mask[t] != 0;
+            a.nreal[chunk0 + cl] = n;
+        }
     if (!a.fuse_scan) return;
     // last-CTA-done: the CTA that completes the arrival count runs the scan on
     // everyone's partials (fences order the partial stores before the count)

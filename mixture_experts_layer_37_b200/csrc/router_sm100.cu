@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             const int chunk = tile * (RBM / kChunkTokens) + q;
             const int64_t t = (int64_t)chunk * kChunkTokens + lane;
             const bool valid = t < a.T;
+            const bool real = valid && (a.mask == nullptr || a.mask[t] != 0);  // padding selects nothing
             float m = -INFINITY;
 #pragma unroll 1
             for (int e = 0; e < E; ++e) {
@@ -258,25 +259,27 @@ __global__ void __launch_bounds__(kRThreads, 1)
             if (valid) {
 #pragma unroll 1
                 for (int j = 0; j < k; ++j) {
-                    a.topk_idx[t * k + j] = sel[j];
-                    a.topk_w[t * k + j] = row[sel[j]] / psel;
+                    a.topk_idx[t * k + j] = real ? sel[j] : -1;
+                    a.topk_w[t * k + j] = real ? row[sel[j]] / psel : 0.f;
                 }
             }
-            // chunk statistics: fixed-order tree sums in fp64, ballot counts
+            // chunk statistics over the real tokens: fixed-order tree sums in fp64, ballot counts
             if (chunk < a.nchunk) {
 #pragma unroll 1
                 for (int e = 0; e < E; ++e) {
-                    double v = valid ? (double)row[e] : 0.0;
+                    double v = real ? (double)row[e] : 0.0;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                     int cnt = 0;
 #pragma unroll 1
-                    for (int j = 0; j < k; ++j) cnt += __popc(__ballot_sync(0xffffffffu, valid && sel[j] == e));
+                    for (int j = 0; j < k; ++j) cnt += __popc(__ballot_sync(0xffffffffu, real && sel[j] == e));
                     if (lane == 0) {
                         a.psum[(int64_t)e * a.nchunk + chunk] = v;
                         a.hist[(int64_t)e * a.nchunk + chunk] = cnt;
                     }
                 }
+                const int nr = __popc(__ballot_sync(0xffffffffu, real));
+                if (a.mask != nullptr && lane == 0) a.nreal[chunk] = nr;
             }
         }
     }

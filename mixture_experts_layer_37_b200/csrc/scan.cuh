@@ -8,7 +8,8 @@
 // experts, load balancing, capacity factor" (dpshk.com/news/6005940) §2.4;
 // groups per expert as in "Hand-building a LLaMA4-MoE" (dpshk.com/news/
 // 5809432) §2.4) and f_e = n_e/(T*k), p_e = (1/T) sum_t p[t,e],
-// L_aux = alpha*E*sum_e f_e p_e (MoE-basics §2.3, §3.1).
+// L_aux = alpha*E*sum_e f_e p_e (MoE-basics §2.3, §3.1), with T the number of
+// real tokens when padding is masked (LLaMA4-MoE §4.1).
 // Every sum has a fixed order, so results do not depend on scheduling.
 #pragma once
 
@@ -70,12 +71,28 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
         for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
         if (lane == 0) {
             sCount[e] = run;
-            sP[e] = (pp != nullptr && a.T > 0) ? ps / (double)a.T : 0.0;
+            sP[e] = pp != nullptr ? ps : 0.0;  // divided by the real-token count below
             if (a.psum_total != nullptr) a.psum_total[e] = ps;
         }
     }
     __syncthreads();
     if (warp == 0) {
+        // real tokens: every token, or the per-chunk counts of unmasked tokens summed in chunk order
+        int64_t t_real = a.T;
+        if (a.nreal != nullptr) {
+            int64_t run = 0;
+            for (int c0 = 0; c0 < nc; c0 += 32) {
+                int v = c0 + lane < nc ? __ldcg(a.nreal + c0 + lane) : 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                run += v;
+            }
+            t_real = run;
+        }
+        if (lane == 0 && a.shared_off != nullptr) {
+            a.shared_off[0] = 0;
+            a.shared_off[1] = (int32_t)a.T;
+        }
         // kept offsets: exclusive scan of min(n_e, cap) over experts, 32 at a time
         int run = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
@@ -93,10 +110,11 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
             // statistics in a fixed order: lane-strided partial sums, then lane 0 adds them in lane order
             double l = 0.0;
             for (int e = lane; e < E; e += 32) {
-                const double f = a.T > 0 ? (double)sCount[e] / ((double)a.T * a.k) : 0.0;
+                const double f = t_real > 0 ? (double)sCount[e] / ((double)t_real * a.k) : 0.0;
+                const double pe = t_real > 0 ? sP[e] / (double)t_real : 0.0;
                 if (a.f) a.f[e] = (float)f;
-                if (a.p) a.p[e] = (float)sP[e];
-                l += f * sP[e];
+                if (a.p) a.p[e] = (float)pe;
+                l += f * pe;
             }
             double tot = 0.0;
             for (int i = 0; i < 32; ++i) tot += __shfl_sync(0xffffffffu, l, i);

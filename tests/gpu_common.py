@@ -34,10 +34,17 @@ def weights_dev(wl, inp) -> dict:
     w = {"w_router": to_dev(inp["w_router"])}
     if inp.get("router_bias") is not None:
         w["router_bias"] = to_dev(np.asarray(inp["router_bias"], dtype=np.float32))
-    for n in ("w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2"):
+    for n in ("w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2", "shared_gate", "shared_up", "shared_down",
+              "shared_w1", "shared_b1", "shared_w2", "shared_b2"):
         if n in inp:
             w[n] = to_dev(inp[n])
     return w
+
+
+def mask_dev(inp):
+    """The padding mask of the inputs on the device, or None."""
+    m = inp.get("token_mask")
+    return None if m is None else torch.from_numpy(np.ascontiguousarray(m)).cuda()
 
 
 def host_f64(t: torch.Tensor) -> np.ndarray:
@@ -109,4 +116,11 @@ SMALL_WORKLOADS = [
                capacity_factor=0.5, zipf_router_bias=True, seed=107, w_std=0.05),
     W.Workload("e64_k8_f32", T=96, d=32, ffn=48, E=64, k=8, act="swiglu", dtype="f32",
                capacity_factor=0.0, seed=108),
+    # padding mask and shared experts (readings R16, R17)
+    W.Workload("shared2_swiglu_pad", T=700, d=128, ffn=192, E=8, k=2, act="swiglu", dtype="bf16",
+               capacity_factor=1.0, seed=110, n_shared=2, pad_fraction=0.2),
+    W.Workload("shared_gelu_pad", T=333, d=128, ffn=128, E=6, k=2, act="gelu_bias", dtype="bf16",
+               capacity_factor=0.9, seed=111, n_shared=1, pad_fraction=0.3),
+    W.Workload("f32_shared_pad", T=130, d=64, ffn=96, E=4, k=2, act="swiglu", dtype="f32",
+               capacity_factor=1.0, seed=112, n_shared=1, pad_fraction=0.25),
 ]

@@ -41,9 +41,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_config_struct_layout_matches_header():
-    assert ctypes.sizeof(M.MoEConfigC) == 56
-    assert M.MoEConfigC.capacity_factor.offset == 32
-    assert ctypes.sizeof(M.MoEWeightsC) == 7 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
+    assert ctypes.sizeof(M.MoEConfigC) == 64
+    assert M.MoEConfigC.capacity_factor.offset == 32 and M.MoEConfigC.n_shared.offset == 56
+    assert ctypes.sizeof(M.MoEWeightsC) == 12 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
 
 
 @pytest.mark.parametrize("T,k,E,cf", [(64, 2, 4, 1.25), (4096, 2, 8, 1.25), (8192, 2, 8, 1.25), (32768, 2, 32, 1.0),
@@ -109,7 +109,12 @@ def test_invalid_configs_rejected_on_host(lib):
     for name in ("auto", "copy", "gather"):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, dispatch=name).c()
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
-    for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("dispatch", 3), ("dispatch", -1)):
+    assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, n_shared=8).c()),
+                                  ctypes.byref(size)) == M.MOE_OK
+    assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, n_shared=9).c()),
+                                  ctypes.byref(size)) == M.MOE_ERR_UNSUPPORTED
+    for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("dispatch", 3), ("dispatch", -1), ("n_shared", -1),
+                     ("reserved", 1)):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
         setattr(cfg, field, v)
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
@@ -122,27 +127,34 @@ def test_null_and_workspace_errors_launch_nothing(lib):
     c = cfg.c()
     w = M.MoEWeightsC()
     o = M.MoEOutputsC()
-    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), None, None, ctypes.byref(o), None, 0, None) == \
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), None, None, None, ctypes.byref(o), None, 0, None) == \
         M.MOE_ERR_INVALID_ARG
-    assert lib.moe_forward(ctypes.byref(c), None, None, None, None, None, 0, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(ctypes.byref(c), None, None, None, None, None, None, 0, None) == M.MOE_ERR_INVALID_ARG
     # well-formed pointers (never dereferenced) but no workspace
     fake = ctypes.c_void_p(1 << 40)
-    w = M.MoEWeightsC(fake, None, fake, fake, fake, None, None)
+    w = M.MoEWeightsC(fake, None, fake, fake, fake, None, None, None, None, None, None, None)
     o = M.MoEOutputsC(*([fake] * 10 + [None, None]))
-    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, ctypes.byref(o), None, 0, None) == \
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, None, ctypes.byref(o), None, 0, None) == \
         M.MOE_ERR_WORKSPACE
     need = M.moe_workspace_size(cfg)
-    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, ctypes.byref(o), fake, need - 1, None) == \
-        M.MOE_ERR_WORKSPACE
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), fake, None, None, ctypes.byref(o), fake, need - 1,
+                           None) == M.MOE_ERR_WORKSPACE
     # misaligned activation pointer
     mis = ctypes.c_void_p((1 << 40) + 8)
-    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), mis, None, ctypes.byref(o), fake, need, None) == \
+    assert lib.moe_forward(ctypes.byref(c), ctypes.byref(w), mis, None, None, ctypes.byref(o), fake, need, None) == \
         M.MOE_ERR_INVALID_ARG
+    # shared experts without their weights
+    cs = M.MoEConfig(T=128, d=128, ffn=128, E=8, k=2, n_shared=1)
+    need_s = M.moe_workspace_size(cs)
+    assert need_s > need
+    assert lib.moe_forward(ctypes.byref(cs.c()), ctypes.byref(w), fake, None, None, ctypes.byref(o), fake, need_s,
+                           None) == M.MOE_ERR_INVALID_ARG
+    assert M.moe_forward_launch_count(cs) == 7
     # swiglu without w_up
-    w2 = M.MoEWeightsC(fake, None, fake, None, fake, None, None)
+    w2 = M.MoEWeightsC(fake, None, fake, None, fake, None, None, None, None, None, None, None)
     assert lib.moe_expert_ffn(ctypes.byref(c), ctypes.byref(w2), fake, fake, fake, fake, need, None) == \
         M.MOE_ERR_INVALID_ARG
-    assert lib.moe_router_topk(ctypes.byref(c), fake, fake, None, None, None, fake, None, None, fake, need,
+    assert lib.moe_router_topk(ctypes.byref(c), fake, fake, None, None, None, None, fake, None, None, fake, need,
                                None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(ctypes.byref(c), None, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_aux_stats(ctypes.byref(c), None, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG

@@ -12,7 +12,7 @@ import torch
 import mixture_experts_layer_37_b200 as M
 import workloads as W
 from oracle import moe_oracle as O
-from gpu_common import (SMALL_WORKLOADS, expert_rows_ref, host_f64, logit_error_bound, out_close, rel_close,
+from gpu_common import (SMALL_WORKLOADS, expert_rows_ref, host_f64, logit_error_bound, mask_dev, out_close, rel_close,
                         sample_tokens, to_dev, weights_dev)
 
 pytestmark = pytest.mark.gpu
@@ -36,12 +36,15 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     dev = lambda a: to_dev(np.ascontiguousarray(a))  # noqa: E731
     R = int(r["offsets"][-1])
     rows_cap = M.moe_max_rows(cfg)
+    tm = mask_dev(inp)
+    real = np.ones(T, dtype=bool) if tm is None else inp["token_mask"] != 0
 
     # ---- 1. router + softmax + top-k with identical logits: bit-exact indices
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
     tw = torch.empty((T, k), dtype=torch.float32, device="cuda")
     probs = torch.empty((T, E), dtype=torch.float32, device="cuda")
-    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), dev(feed), idx, tw, None, probs, ws)
+    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), dev(feed), idx, tw, None, probs, ws,
+                      token_mask=tm)
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), r["idx"]), "top-k indices differ on identical logits"
     ok, worst = rel_close(tw.cpu().numpy(), r["w"])
@@ -53,21 +56,22 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     #         the chosen experts are the top-k of the GPU's own logits, and equal
     #         the oracle's wherever the oracle's k-th / (k+1)-th gap exceeds the bound
     lo = torch.empty((T, E), dtype=torch.float32, device="cuda")
-    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), None, idx, tw, lo, probs, ws)
+    M.moe_router_topk(cfg, x, wd["w_router"], wd.get("router_bias"), None, idx, tw, lo, probs, ws, token_mask=tm)
     torch.cuda.synchronize()
     lg = lo.cpu().numpy().astype(np.float64)
     gi = idx.cpu().numpy()
+    assert (gi[~real] == -1).all() and (tw.cpu().numpy()[~real] == 0).all(), "padding selected an expert"
     # the GPU's probabilities and weights are the softmax / renormalisation of its own logits
     pg = probs.cpu().numpy().astype(np.float64)
     z = np.exp(lg - lg.max(axis=1, keepdims=True))
     assert rel_close(pg, z / z.sum(axis=1, keepdims=True), rtol=1e-5, atol=1e-12)[0]
-    sel = np.take_along_axis(pg, gi.astype(np.int64), axis=1)
-    assert rel_close(tw.cpu().numpy(), sel / sel.sum(axis=1, keepdims=True), rtol=1e-5)[0]
+    sel = np.take_along_axis(pg[real], gi[real].astype(np.int64), axis=1)
+    assert rel_close(tw.cpu().numpy()[real], sel / sel.sum(axis=1, keepdims=True), rtol=1e-5)[0]
     toks = np.arange(T) if T <= 8192 else np.random.default_rng(1).choice(T, 8192, replace=False)
     bound = logit_error_bound(wl, inp, toks)
     err = np.abs(lg[toks] - r["logits64"][toks])
     assert (err <= bound).all(), f"router logits error {err.max()} above bound"
-    for t in range(T):
+    for t in np.nonzero(real)[0]:
         sel = set(gi[t].tolist())
         for j, e in enumerate(gi[t]):
             for u in range(E):
@@ -80,7 +84,7 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     gap = srt[:, k - 1] - (srt[:, k] if k < E else -np.inf)
     full_bound = logit_error_bound(wl, inp, np.arange(T)) if T <= 8192 else None
     margin = 2 * (full_bound.max(axis=1) if full_bound is not None else bound.max())
-    clear = gap > margin
+    clear = (gap > margin) & real
     assert np.array_equal(np.sort(gi[clear], axis=1), np.sort(r["idx"][clear], axis=1))
 
     # ---- 3. dispatch with identical indices: bit-exact counts/offsets/slots/permutation, exact row copies
@@ -156,7 +160,7 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
 
     # ---- 7. whole forward, logits fed: bit-exact routing/dispatch, outputs within tolerance
     layer = M.MoELayer(cfg, wd)
-    o = layer.forward(x, logits_in=dev(feed))
+    o = layer.forward(x, logits_in=dev(feed), token_mask=tm)
     layer.check()
     assert np.array_equal(o["topk_idx"].cpu().numpy(), r["idx"])
     assert np.array_equal(o["counts"].cpu().numpy(), r["counts"])
@@ -175,7 +179,7 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     first = {n: v.clone() for n, v in o.items()}
 
     # ---- 8. determinism: a second run is bit-identical
-    o2 = layer.forward(x, logits_in=dev(feed))
+    o2 = layer.forward(x, logits_in=dev(feed), token_mask=tm)
     torch.cuda.synchronize()
     for n, v in first.items():
         a, b = v.cpu(), o2[n].cpu()
@@ -184,7 +188,7 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
         assert torch.equal(a, b), f"{n} differs between two identical runs"
 
     # ---- 9. whole forward with the GPU's own router: same outputs where routing agrees
-    o3 = layer.forward(x)
+    o3 = layer.forward(x, token_mask=tm)
     layer.check()
     gi = o3["topk_idx"].cpu().numpy()
     gs = o3["slot"].cpu().numpy()
@@ -329,3 +333,12 @@ def test_gather_dispatch_equals_copy(wl):
             if n == "src_assign":
                 a, b = a[:R], b[:R]
             assert torch.equal(a, b), f"{key}: {n} differs"
+
+
+# the llama4moe layer with one shared expert and 10 % padding, at full size
+SHARED_FULL = W.WORKLOADS["llama4moe_t4096"].with_(name="llama4moe_t4096_shared1_pad10", n_shared=1, pad_fraction=0.1)
+
+
+@pytest.mark.parametrize("gemm", ["auto", "cta_pair"])
+def test_shared_experts_and_padding_full_size(gemm):
+    _check_workload(SHARED_FULL, full_size=True, gemm=gemm)
