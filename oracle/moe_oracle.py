@@ -39,6 +39,13 @@ DESIGN.md):
       weight 0, no dispatch, no routed output) and is left out of f and p,
       which divide by the number of real tokens T_real; the capacity stays
       ceil(T*k/E * cf) of the whole batch T.  T_real = 0 gives zero statistics.
+  R18 INT8 expert weights (the long-context MoE page, §3: INT8 weights times
+      a scale computed per expert and per dimension, dequantised for use):
+      per expert and output column n, scale s = max_k |W[k,n]| / 127 and code
+      q = clamp(rint(W / s), -127, 127) (ties to even), both in fp32, the
+      precision the library takes the decision in (an all-zero column has
+      s = 0, q = 0); the layer then runs on the dequantised weights q * s.
+      Shared experts keep their native weights.
   R17 shared experts ([LLaMA4-MoE] §5.2: fixed experts take part in every
       token's computation): n_shared experts of the routed experts' form, own
       weights, applied to every token (padding included) with weight 1 and
@@ -271,9 +278,36 @@ def route(wl, inputs: dict, logits_feed: Optional[np.ndarray] = None) -> dict:
             "f": f, "p_mean": pm, "l_aux": laux, "t_real": int(real.sum()), **disp}
 
 
+def quantize_int8(w: np.ndarray) -> tuple:
+    """Reading R18: per-output-channel symmetric INT8 codes of one expert's
+    matrix w [K, N] (float32 values): s[n] = max_k |w[k,n]| / 127 and
+    q = clamp(rint(w / s), -127, 127), all in float32; s = 0 gives q = 0."""
+    w = np.asarray(w, dtype=np.float32)
+    amax = np.abs(w).max(axis=0).astype(np.float32)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint((w / safe[None, :]).astype(np.float32))
+    q = np.clip(q, -127, 127)
+    q = np.where(s[None, :] > 0, q, 0).astype(np.int8)
+    return q, s
+
+
+def dequantize_int8(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """Reading R18: the weights the INT8 layer uses, q * s (float64)."""
+    return q.astype(np.float64) * s.astype(np.float64)[None, :]
+
+
 def expert_weights_f64(wl, inputs: dict, e: int) -> tuple:
-    """Expert e's parameters decoded to float64."""
+    """Expert e's parameters decoded to float64 (dequantised INT8 weights when
+    the workload stores its routed experts in INT8, reading R18)."""
     dt = wl.dtype
+    if getattr(wl, "weights", "native") == "int8":
+        def dq(name):
+            q, s = quantize_int8(to_f64(inputs[name][e], dt).astype(np.float32))
+            return dequantize_int8(q, s)
+        if wl.act == "swiglu":
+            return (dq("w_gate"), dq("w_up"), dq("w_down"))
+        return (dq("w1"), to_f64(inputs["b1"][e], dt), dq("w2"), to_f64(inputs["b2"][e], dt))
     if wl.act == "swiglu":
         return (to_f64(inputs["w_gate"][e], dt), to_f64(inputs["w_up"][e], dt), to_f64(inputs["w_down"][e], dt))
     return (to_f64(inputs["w1"][e], dt), to_f64(inputs["b1"][e], dt),

@@ -424,12 +424,49 @@ def check_shared_experts(o):
         np.testing.assert_allclose(pad["out"], ffn(sh).numpy(), rtol=1e-12, atol=1e-12)
 
 
+def check_int8_quantization(o):
+    """Reading R18 (INT8 weights with a per-expert, per-dimension scale, the
+    long-context MoE page §3): hand codes, the half-step error bound
+    |w - q*s| <= s/2, exact recovery of matrices already on the code grid,
+    codes within [-127, 127] with +-127 reached in every non-zero column, an
+    all-zero column, and the layer on int8 weights equal to the layer on the
+    dequantised weights."""
+    w = np.array([[127.0, 0.0, 1.0], [-63.5, 0.0, -0.25], [0.4, 0.0, 0.5]], dtype=np.float32)
+    q, s = o.quantize_int8(w)
+    assert s.tolist() == [np.float32(1.0), 0.0, np.float32(1.0) / np.float32(127.0)]
+    assert q[:, 0].tolist() == [127, -64, 0]          # -63.5 rounds to the even -64
+    assert q[:, 1].tolist() == [0, 0, 0]
+    assert q[0, 2] == 127 and q[2, 2] == 64           # 0.5 * 127 = 63.5 -> 64 (even)
+    rng = np.random.default_rng(4)
+    w = (rng.normal(size=(64, 48)) * rng.uniform(0.01, 3.0, size=(1, 48))).astype(np.float32)
+    q, s = o.quantize_int8(w)
+    assert q.dtype == np.int8 and np.abs(q.astype(int)).max() <= 127
+    assert (np.abs(q.astype(int)).max(axis=0) == 127).all()
+    err = np.abs(w.astype(np.float64) - o.dequantize_int8(q, s))
+    assert (err <= s.astype(np.float64)[None, :] * (0.5 + 1e-6)).all()
+    grid = o.dequantize_int8(q, s).astype(np.float32)
+    q2, s2 = o.quantize_int8(grid)
+    np.testing.assert_array_equal(q2, q)
+    np.testing.assert_allclose(o.dequantize_int8(q2, s2), grid, rtol=1e-6)
+    # the layer on int8 weights is the layer on the dequantised weights
+    wl = _wl(T=19, d=16, ffn=24, E=2, k=1, act="swiglu", capacity_factor=0.0, weights="int8")
+    inp = W.make_inputs(wl.with_(weights="native", seed=8))
+    deq = {}
+    for n in ("w_gate", "w_up", "w_down"):
+        deq[n] = np.stack([o.dequantize_int8(*o.quantize_int8(inp[n][e].astype(np.float32))) for e in range(2)])
+    a = o.forward(wl, inp)
+    # (the f32 workload's inputs are read as float32, so the dequantised weights pass through one fp32 rounding)
+    b = o.forward(wl.with_(weights="native"), {**inp, **{n: v.astype(np.float32) for n, v in deq.items()}})
+    assert np.abs(a["out"] - b["out"]).max() <= 1e-6 * np.abs(b["out"]).max()
+    assert np.abs(a["out"] - o.forward(wl.with_(weights="native"), inp)["out"]).max() > 1e-9  # quantisation shows
+
+
 CHECKS = [check_worked_example, check_uniform_alpha, check_sums_to_one, check_topk_bruteforce,
           check_tie_lower_id, check_renorm_is_selected_softmax, check_softmax_closed_form,
           check_capacity, check_dispatch_hand_case, check_dispatch_bruteforce,
           check_activation_closed_forms, check_dense_reduction, check_teaching_layer,
           check_combine_properties, check_drop_path_end_to_end, check_empty, check_padding_mask,
-          check_shared_experts]
+          check_shared_experts, check_int8_quantization]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
@@ -534,7 +571,24 @@ def _shared_averaged(wl, inputs, xr):
     return acc / max(wl.n_shared, 1)
 
 
+def _quant_global_scale(w):
+    w = np.asarray(w, dtype=np.float32)
+    s = np.full(w.shape[1], np.abs(w).max() / np.float32(127.0), dtype=np.float32)
+    q = np.clip(np.rint(w / s[None, :]), -127, 127).astype(np.int8)
+    return q, s
+
+
+def _quant_truncating(w):
+    w = np.asarray(w, dtype=np.float32)
+    s = (np.abs(w).max(axis=0) / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0))
+    q = np.where(s[None, :] > 0, np.clip(np.trunc(w / safe[None, :]), -127, 127), 0).astype(np.int8)
+    return q, s
+
+
 MUTANTS = {
+    "int8_global_scale": dict(quantize_int8=_quant_global_scale),
+    "int8_truncating_codes": dict(quantize_int8=_quant_truncating),
     "padding_selects_experts": dict(mask_padding=_mask_ignored),
     "padding_counted_in_stats": dict(real_tokens=_stats_over_all_tokens),
     "shared_experts_averaged": dict(shared_outputs=_shared_averaged),

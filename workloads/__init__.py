@@ -107,6 +107,7 @@ class Workload:
     seed: int = 0
     n_shared: int = 0         # always-on shared experts (same FFN form as the routed ones)
     pad_fraction: float = 0.0  # expected fraction of padding tokens (token_mask = 0)
+    weights: str = "native"   # routed experts' weights: "native" (the dtype) or "int8" (quantised by the layer)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
