@@ -57,6 +57,7 @@ def parse():
     ap.add_argument("--dispatch", default="auto", choices=["auto", "copy", "gather"])
     ap.add_argument("--n-shared", type=int, default=None, help="shared experts (default: the workload's)")
     ap.add_argument("--pad-fraction", type=float, default=None, help="padding tokens (default: the workload's)")
+    ap.add_argument("--weights", default=None, choices=["native", "int8"], help="routed experts' weight storage")
     return ap.parse_args()
 
 
@@ -196,6 +197,8 @@ def run_native(a):
         wl = wl.with_(n_shared=a.n_shared)
     if a.pad_fraction is not None:
         wl = wl.with_(pad_fraction=a.pad_fraction)
+    if a.weights is not None:
+        wl = wl.with_(weights=a.weights)
     cfg = M.MoEConfig.of(wl, a.router_kernel, a.gemm_kernel, a.dispatch)
     seed = wl.seed + 1000 * rank
     inp = W.make_inputs(wl, seed=seed)
@@ -210,6 +213,9 @@ def run_native(a):
     weights = {n: dev(inp[n]) for n in wnames if n in inp}
     if inp.get("router_bias") is not None:
         weights["router_bias"] = dev(np.asarray(inp["router_bias"], dtype=np.float32))
+    if wl.weights == "int8":
+        weights = M.quantize_expert_weights(cfg, weights)  # once, before anything is timed
+        torch.cuda.synchronize()
     x = dev(inp["x"])
     tmask = dev(inp["token_mask"]) if "token_mask" in inp else None
     layer = M.MoELayer(cfg, weights)
@@ -292,11 +298,23 @@ def run_native(a):
     bpe = 2 if wl.dtype == "bf16" else 4
     gemm1_flops = (4 if wl.act == "swiglu" else 2) * wl.d * wl.ffn * R
     gemm2_flops = 2 * wl.d * wl.ffn * R
+    # each expert GEMM is bound by the tensor cores or by streaming the weights of
+    # the experts that received rows, whichever its FLOP per byte puts it under
+    hit = int((layer.outputs["offsets"].diff() > 0).sum().item())
+    wbpe = 1 if wl.weights == "int8" else bpe
+    nmat1 = 2 if wl.act == "swiglu" else 1
+    gemm1_bytes = hit * nmat1 * wl.d * wl.ffn * wbpe + R * (wl.d + wl.ffn) * bpe
+    gemm2_bytes = hit * wl.d * wl.ffn * wbpe + R * (wl.d + wl.ffn) * bpe
+    balance = pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+
+    def gemm_bound(flops, nbytes):
+        return ("tensor", flops) if flops / nbytes >= balance else ("hbm", nbytes)
+
     algo = {
         "router": ("hbm", wl.T * wl.d * bpe + wl.d * wl.E * bpe + wl.T * wl.k * 8),
         "scatter": ("hbm", 2 * R * wl.d * bpe + wl.T * wl.k * 4 * 3),
-        "gemm1": ("tensor", gemm1_flops),
-        "gemm2": ("tensor", gemm2_flops),
+        "gemm1": gemm_bound(gemm1_flops, gemm1_bytes),
+        "gemm2": gemm_bound(gemm2_flops, gemm2_bytes),
         "combine": ("hbm", R * wl.d * bpe + (1 + wl.n_shared) * wl.T * wl.d * bpe + wl.T * wl.k * 8),
     }
     for i in range(wl.n_shared):
@@ -314,10 +332,10 @@ def run_native(a):
         achieved = work / dur_s / 1e9
         peak = pk["hbm_gbs"]
         unit = "GB/s"
-    roofline = {"bound": bound, "kernel": f"grouped_gemm_kernel ({dname})" if bound == "tensor" else dname,
+    roofline = {"bound": bound, "kernel": f"grouped expert GEMM ({dname})" if "gemm" in dname else dname,
                 "achieved": round(achieved, 2), "peak": peak, "peak_source": f"{pk_src} ({'bf16 dense burst' if bound == 'tensor' else 'HBM copy'})",
                 "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": recorded_traffic(dname, a.workload) if bound == "tensor" else None}
+                "traffic": recorded_traffic(dname, a.workload) if "gemm" in dname and wl.weights == "native" else None}
     stages = {}
     for j, n in enumerate(names):
         b, w = algo[n]

@@ -106,6 +106,16 @@ typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_ONE_CTA = 1, MOE_GEMM_CTA_PAIR = 2 } 
  *                        src_assign, and x_perm is never written. */
 typedef enum { MOE_DISPATCH_AUTO = 0, MOE_DISPATCH_COPY = 1, MOE_DISPATCH_GATHER = 2 } moe_dispatch_mode_t;
 
+/* Storage of the routed experts' weights.
+ *   MOE_WEIGHTS_NATIVE  the config's dtype;
+ *   MOE_WEIGHTS_INT8    INT8 codes with a per-expert, per-output-column fp32
+ *                       scale (from moe_quantize_int8; the long-context MoE
+ *                       page §3): the layer uses the weights codes * scale.
+ *                       bf16 activations only.  Built for decode-sized batches
+ *                       (a few rows per expert): it halves the weight bytes the
+ *                       FFNs stream.  Shared experts keep native weights. */
+typedef enum { MOE_WEIGHTS_NATIVE = 0, MOE_WEIGHTS_INT8 = 1 } moe_weight_format_t;
+
 /* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
  * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
 typedef struct {
@@ -122,7 +132,7 @@ typedef struct {
     int32_t gemm_kernel;       /* moe_gemm_kernel_t (0: library's choice) */
     int32_t dispatch;          /* moe_dispatch_mode_t (0: library's choice) */
     int32_t n_shared;          /* shared experts, 0..8 (LLaMA4-MoE §5.2; see moe_forward) */
-    int32_t reserved;          /* must be 0 */
+    int32_t weight_format;     /* moe_weight_format_t of the routed experts */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */
@@ -140,6 +150,10 @@ typedef struct {
     const void* shared_down_or_w2;   /* [S, ffn, d] */
     const void* shared_b1;           /* [S, ffn] GELU only, else NULL */
     const void* shared_b2;           /* [S, d]   GELU only, else NULL */
+    /* MOE_WEIGHTS_INT8: w_gate_or_w1 / w_up / w_down_or_w2 hold int8 codes and these their scales */
+    const float* gate_or_w1_scale;   /* [E, ffn] */
+    const float* up_scale;           /* [E, ffn] SwiGLU only, else NULL */
+    const float* down_or_w2_scale;   /* [E, d] */
 } moe_weights_t;
 
 /* Outputs of moe_forward (device).  R_max = moe_max_rows(). */
@@ -194,6 +208,16 @@ moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void*
                              const float* logit_bias, const float* logits_in, const uint8_t* token_mask,
                              int32_t* topk_idx, float* topk_w, float* logits_out, float* probs_out,
                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Quantise expert weights w [E, K, N] (config dtype, on the device) to INT8
+ * codes q [E, K, N] (int8) and scales scale [E, N] (float32), per expert and
+ * output column n: scale = max_k |w[e,k,n]| / 127, q = clamp(rint(w / scale),
+ * -127, 127), ties to even, all in fp32; an all-zero column gets scale 0 and
+ * codes 0 (the long-context MoE page §3: a scale per expert and per
+ * dimension).  For SwiGLU call it for W_gate and W_up (K = d, N = ffn) and
+ * W_down (K = ffn, N = d).  Asynchronous on `stream`. */
+moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
+                               cudaStream_t stream);
 
 /* Capacity-bounded dispatch (MoE-basics §2.4; LLaMA4-MoE §2.4).
  *   topk_idx [T,k] int32 in [0,E), or -1 (selects nothing: padding).

@@ -43,13 +43,14 @@ class MoEConfigC(ctypes.Structure):
                 ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("router_kernel", ctypes.c_int32),
                 ("gemm_kernel", ctypes.c_int32), ("dispatch", ctypes.c_int32), ("n_shared", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("weight_format", ctypes.c_int32)]
 
 
 class MoEWeightsC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_router", "router_logit_bias", "w_gate_or_w1", "w_up", "w_down_or_w2", "b1", "b2",
-                 "shared_gate_or_w1", "shared_up", "shared_down_or_w2", "shared_b1", "shared_b2")]
+                 "shared_gate_or_w1", "shared_up", "shared_down_or_w2", "shared_b1", "shared_b2",
+                 "gate_or_w1_scale", "up_scale", "down_or_w2_scale")]
 
 
 class MoEOutputsC(ctypes.Structure):
@@ -109,7 +110,7 @@ EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_wo
                     "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled",
                     "moe_dispatch_noalloc", "moe_dp_workspace_size", "moe_dp_max_rows", "moe_dp_route",
                     "moe_dp_finish", "moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_wait",
-                    "moe_pipeline_check", "moe_pipeline_destroy")
+                    "moe_pipeline_check", "moe_pipeline_destroy", "moe_quantize_int8")
 
 
 # ---------------------------------------------------------------- config
@@ -128,13 +129,15 @@ class MoEConfig:
     gemm_kernel: str = "auto"    # "auto" | "one_cta" | "cta_pair"
     dispatch: str = "auto"       # "auto" | "copy" | "gather"
     n_shared: int = 0            # shared experts, applied to every token with weight 1
+    weights: str = "native"      # routed experts' weights: "native" (the dtype) or "int8" (codes + scales)
 
     def c(self) -> MoEConfigC:
         return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
                           MOE_DT_BF16 if self.dtype == "bf16" else MOE_DT_F32,
                           MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
                           float(self.capacity_factor), float(self.aux_alpha), ROUTER_KERNELS[self.router_kernel],
-                          GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch], int(self.n_shared), 0)
+                          GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch], int(self.n_shared),
+                          1 if self.weights == "int8" else 0)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -144,7 +147,8 @@ class MoEConfig:
     def of(wl, router_kernel: str = "auto", gemm_kernel: str = "auto", dispatch: str = "auto") -> "MoEConfig":
         """From a workload description (anything with the same field names)."""
         return MoEConfig(wl.T, wl.d, wl.ffn, wl.E, wl.k, wl.dtype, wl.act, wl.capacity_factor, wl.aux_alpha,
-                         router_kernel, gemm_kernel, dispatch, getattr(wl, "n_shared", 0))
+                         router_kernel, gemm_kernel, dispatch, getattr(wl, "n_shared", 0),
+                         getattr(wl, "weights", "native"))
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -223,7 +227,9 @@ def _weights_c(w: dict) -> MoEWeightsC:
     return MoEWeightsC(g("w_router"), g("router_bias"), g("w_gate") if "w_gate" in w else g("w1"), g("w_up"),
                        g("w_down") if "w_down" in w else g("w2"), g("b1"), g("b2"),
                        g("shared_gate") if "shared_gate" in w else g("shared_w1"), g("shared_up"),
-                       g("shared_down") if "shared_down" in w else g("shared_w2"), g("shared_b1"), g("shared_b2"))
+                       g("shared_down") if "shared_down" in w else g("shared_w2"), g("shared_b1"), g("shared_b2"),
+                       g("w_gate_scale") if "w_gate_scale" in w else g("w1_scale"), g("w_up_scale"),
+                       g("w_down_scale") if "w_down_scale" in w else g("w2_scale"))
 
 
 def moe_expert_ffn(cfg: MoEConfig, weights: dict, x_perm, offsets, y_perm, ws: Workspace, stream=None) -> None:
@@ -481,3 +487,29 @@ class Pipeline:
             self.close()
         except Exception:
             pass
+
+
+def moe_quantize_int8(cfg: MoEConfig, w: torch.Tensor, stream=None):
+    """INT8 codes and per-expert, per-output-column scales of expert weights
+    w [E, K, N] (moe_quantize_int8).  Returns (codes int8 [E, K, N], scales
+    float32 [E, N]), both on w's device."""
+    L = lib()
+    f = L.moe_quantize_int8
+    f.argtypes = [_CFG, _P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]
+    f.restype = ctypes.c_int
+    E, K, N = w.shape
+    q = torch.empty((E, K, N), dtype=torch.int8, device=w.device)
+    s = torch.empty((E, N), dtype=torch.float32, device=w.device)
+    _check(f(ctypes.byref(cfg.c()), _ptr(w), int(K), int(N), _ptr(q), _ptr(s), _stream(stream)), "moe_quantize_int8")
+    return q, s
+
+
+def quantize_expert_weights(cfg: MoEConfig, weights: dict, stream=None) -> dict:
+    """A copy of `weights` whose routed experts are stored as INT8 codes plus
+    scales (w_gate/w_up/w_down or w1/w2 replaced by codes, with *_scale added)."""
+    out = dict(weights)
+    for name in (("w_gate", "w_up", "w_down") if cfg.act == "swiglu" else ("w1", "w2")):
+        q, s = moe_quantize_int8(cfg, weights[name], stream)
+        out[name] = q
+        out[name + "_scale"] = s
+    return out

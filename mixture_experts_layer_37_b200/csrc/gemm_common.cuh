@@ -162,6 +162,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tbas
 // box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch, uint32_t box_inner,
               uint32_t box_outer);
+// The same for any element type, without swizzle (rows land in shared memory as they are in memory).
+bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t pitch, uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace gemm
 }  // namespace moe

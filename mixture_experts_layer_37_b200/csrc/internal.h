@@ -130,12 +130,21 @@ struct FfnArgs {
     const void* gather_x = nullptr;    // [T, d] or null
     const int32_t* src_assign = nullptr;
     int k = 0;
+    // INT8 weights (w1 / w_up / w2 hold codes): per-expert, per-output-column scales
+    bool int8 = false;
+    const float* w1_scale = nullptr;   // [E, ffn]
+    const float* w_up_scale = nullptr; // [E, ffn] or null
+    const float* w2_scale = nullptr;   // [E, d]
 };
 // bf16: tcgen05 grouped GEMMs (two launches).  Returns cudaErrorInvalidValue
 // when a tensor map cannot be encoded.
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s);
 // f32: SIMT FMA grouped GEMMs (two launches).
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
+// bf16 activations, INT8 weights (two launches), and the quantiser.
+cudaError_t launch_ffn_int8(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_quantize_int8(const void* w, bool bf16, int64_t E, int64_t K, int64_t N, int8_t* q, float* scale,
+                                 cudaStream_t s);
 
 cudaError_t launch_selftest_wait(DevStatus st, cudaStream_t s);
 

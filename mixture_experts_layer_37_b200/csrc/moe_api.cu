@@ -49,9 +49,11 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
         c->router_kernel > MOE_ROUTER_TCGEN05 || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
-        c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER || c->n_shared < 0 || c->reserved != 0)
+        c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER || c->n_shared < 0 ||
+        c->weight_format < MOE_WEIGHTS_NATIVE || c->weight_format > MOE_WEIGHTS_INT8)
         return MOE_ERR_INVALID_ARG;
     if (c->n_shared > kMaxShared) return MOE_ERR_UNSUPPORTED;
+    if (c->weight_format == MOE_WEIGHTS_INT8 && c->dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED;
     if (c->router_kernel == MOE_ROUTER_TCGEN05 &&
         (c->dtype != MOE_DT_BF16 || c->E % 8 != 0 || c->d % 64 != 0))
         return MOE_ERR_UNSUPPORTED;
@@ -183,6 +185,10 @@ moe_status_t check_weights(const moe_config_t* c, const moe_weights_t* w, bool n
             if (w->b1 == nullptr || w->b2 == nullptr || !aligned16(w->b1) || !aligned16(w->b2))
                 return MOE_ERR_INVALID_ARG;
         }
+        if (c->weight_format == MOE_WEIGHTS_INT8 &&
+            (w->gate_or_w1_scale == nullptr || w->down_or_w2_scale == nullptr ||
+             (c->act == MOE_ACT_SWIGLU && w->up_scale == nullptr)))
+            return MOE_ERR_INVALID_ARG;
         if (c->n_shared > 0) {
             if (w->shared_gate_or_w1 == nullptr || w->shared_down_or_w2 == nullptr ||
                 !aligned16(w->shared_gate_or_w1) || !aligned16(w->shared_down_or_w2))
@@ -276,8 +282,10 @@ moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* id
 }
 
 // Whether moe_forward / moe_dp_finish gather the first GEMM's rows from x
-// (on request only: the copy is faster end to end on B200).
-bool gathers(const moe_config_t* c) { return c->dtype == MOE_DT_BF16 && c->dispatch == MOE_DISPATCH_GATHER; }
+// (on request only: the copy is faster end to end on B200; never with INT8 weights).
+bool gathers(const moe_config_t* c) {
+    return c->dtype == MOE_DT_BF16 && c->dispatch == MOE_DISPATCH_GATHER && c->weight_format == MOE_WEIGHTS_NATIVE;
+}
 
 moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* x_perm, const int32_t* offsets,
                      void* y_perm, void* ws, const Plan& pl, cudaStream_t s, cudaEvent_t between = nullptr,
@@ -303,6 +311,16 @@ moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* 
     f.gather_x = gather_x;
     f.src_assign = src_assign;
     f.k = c->k;
+    if (c->weight_format == MOE_WEIGHTS_INT8) {
+        // INT8 routed experts: rows always come from the sorted copy
+        if (x_perm == nullptr) return MOE_ERR_INVALID_ARG;
+        f.int8 = true;
+        f.gather_x = nullptr;
+        f.w1_scale = w->gate_or_w1_scale;
+        f.w_up_scale = w->up_scale;
+        f.w2_scale = w->down_or_w2_scale;
+        return from_cuda(launch_ffn_int8(f, s));
+    }
     return from_cuda(c->dtype == MOE_DT_BF16 ? launch_ffn_bf16_sm100(f, s) : launch_ffn_f32(f, s));
 }
 
@@ -417,6 +435,15 @@ moe_status_t moe_router_topk(const moe_config_t* cfg, const void* x, const void*
     if (cfg->T == 0) return MOE_OK;
     return run_router(cfg, x, w_router, logit_bias, logits_in, token_mask, topk_idx, topk_w, logits_out, probs_out, ws,
                       pl, stream);
+}
+
+moe_status_t moe_quantize_int8(const moe_config_t* cfg, const void* w, int64_t K, int64_t N, int8_t* q, float* scale,
+                               cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if (K <= 0 || N <= 0 || N % 4 != 0) return MOE_ERR_INVALID_ARG;
+    if (w == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_quantize_int8(w, cfg->dtype == MOE_DT_BF16, cfg->E, K, N, q, scale, stream));
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,

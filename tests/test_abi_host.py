@@ -43,7 +43,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_config_struct_layout_matches_header():
     assert ctypes.sizeof(M.MoEConfigC) == 64
     assert M.MoEConfigC.capacity_factor.offset == 32 and M.MoEConfigC.n_shared.offset == 56
-    assert ctypes.sizeof(M.MoEWeightsC) == 12 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
+    assert ctypes.sizeof(M.MoEWeightsC) == 15 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
 
 
 @pytest.mark.parametrize("T,k,E,cf", [(64, 2, 4, 1.25), (4096, 2, 8, 1.25), (8192, 2, 8, 1.25), (32768, 2, 32, 1.0),
@@ -113,8 +113,13 @@ def test_invalid_configs_rejected_on_host(lib):
                                   ctypes.byref(size)) == M.MOE_OK
     assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, n_shared=9).c()),
                                   ctypes.byref(size)) == M.MOE_ERR_UNSUPPORTED
+    assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, weights="int8").c()),
+                                  ctypes.byref(size)) == M.MOE_OK
+    assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, dtype="f32",
+                                                           weights="int8").c()), ctypes.byref(size)) == \
+        M.MOE_ERR_UNSUPPORTED
     for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("dispatch", 3), ("dispatch", -1), ("n_shared", -1),
-                     ("reserved", 1)):
+                     ("weight_format", 2), ("weight_format", -1)):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
         setattr(cfg, field, v)
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG

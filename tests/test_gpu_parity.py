@@ -31,6 +31,8 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     r = O.route(wl, inp)
     feed = r["logits"].astype(np.float32)
     wd = weights_dev(wl, inp)
+    if wl.weights == "int8":
+        wd = M.quantize_expert_weights(cfg, wd)
     x = to_dev(inp["x"])
     ws = M.Workspace(cfg)
     dev = lambda a: to_dev(np.ascontiguousarray(a))  # noqa: E731
