@@ -38,7 +38,7 @@ constexpr int kLStride = kMaxExperts + 1;
 constexpr int kSlabBytes = 32 * 1024;  // one of the two router-weight slab buffers
 constexpr int kMaxTpc = 64;
 constexpr int kSplits = 4;  // K partial sums per token, always (batch-invariant logits)
-constexpr int kBatch = 4;  // 32-column blocks of x loaded per batch
+constexpr int kBatch = 8;  // 32-column blocks of x loaded per batch
 
 __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
     uint4 v;
@@ -282,13 +282,10 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
             stage(slab + 1);
         else
             cp_async_commit();  // empty group: keeps "all but the newest group" meaning slab's copies
-        cp_async_wait_prev();
-        __syncthreads();
-        const uint32_t lds_slab = lds_base + (uint32_t)((slab & 1) * kSlabBytes);
         // this warp's 32-row blocks of the slab: ksplit, ksplit + nsplit, ...
         const int nblk = ks / 32;
-        for (int b0 = ksplit; b0 < nblk; b0 += nsplit * kBatch) {
-            uint4 xa[kBatch], xb[kBatch];
+        uint4 xa[kBatch], xb[kBatch];
+        auto load_batch = [&](int b0) {
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int blk = b0 + u * nsplit;
@@ -296,6 +293,14 @@ __global__ void __launch_bounds__(kThreads, 2) router_bf16_kernel(RouterArgs a) 
                 xa[u] = (blk < nblk && v0) ? ldg_stream_128(x0 + kx) : make_uint4(0, 0, 0, 0);
                 xb[u] = (blk < nblk && v1) ? ldg_stream_128(x1 + kx) : make_uint4(0, 0, 0, 0);
             }
+        };
+        // the first batch of token fragments is in flight while the slab lands
+        load_batch(ksplit);
+        cp_async_wait_prev();
+        __syncthreads();
+        const uint32_t lds_slab = lds_base + (uint32_t)((slab & 1) * kSlabBytes);
+        for (int b0 = ksplit; b0 < nblk; b0 += nsplit * kBatch) {
+            if (b0 != ksplit) load_batch(b0);
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int blk = b0 + u * nsplit;
