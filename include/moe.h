@@ -40,7 +40,9 @@
  *     word and returns; moe_check_device_status reports it.
  *   - Results are deterministic: two calls on the same inputs give
  *     bit-identical outputs (no atomics decide any order or sum).
- *   - Calls that share a workspace must not overlap on the GPU.
+ *   - Calls that share a workspace must not overlap on the GPU.  Calls with
+ *     their own workspaces may be issued from several host threads at once
+ *     (the library's per-device one-time setup is thread-safe).
  */
 #ifndef MOE_H_
 #define MOE_H_

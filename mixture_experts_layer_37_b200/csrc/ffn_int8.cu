@@ -277,14 +277,9 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_int8_kernel(const __grid_con
 template <int MODE>
 cudaError_t launch_q(const CUtensorMap& q0, const CUtensorMap& q1, const CUtensorMap& a, const QArgs& p, int E,
                      cudaStream_t s) {
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_int8_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    const cudaError_t err = ensure_smem_attr(attr, ffn_int8_kernel<MODE>, kQSmem);
+    if (err != cudaSuccess) return err;
     dim3 grid((p.N + kQCols - 1) / kQCols, E);
     ffn_int8_kernel<MODE><<<grid, kQThreads, kQSmem, s>>>(q0, q1, a, p);
     return cudaGetLastError();

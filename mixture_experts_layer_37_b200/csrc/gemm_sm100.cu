@@ -323,13 +323,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
+    static std::atomic<EncodeTiledFn> cached{nullptr};
+    EncodeTiledFn fn = cached.load(std::memory_order_acquire);
     if (fn == nullptr) {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+            q == cudaDriverEntryPointSuccess) {
             fn = reinterpret_cast<EncodeTiledFn>(ptr);
+            cached.store(fn, std::memory_order_release);
+        }
     }
     return fn;
 }
@@ -337,15 +340,9 @@ EncodeTiledFn encode_fn() {
 template <int MODE, bool GATHER = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                         int64_t rows_cap, cudaStream_t s) {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, GATHER>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) attr_set[dev] = true;
-    }
+    static std::atomic<bool> attr_set[64];
+    const cudaError_t err = ensure_smem_attr(attr_set, grouped_gemm_kernel<MODE, GATHER>, kSmemBytes);
+    if (err != cudaSuccess) return err;
     const int64_t tiles_upper = (rows_cap / BM + p.E) * (int64_t)p.n_tiles;
     const int grid = (int)min64(tiles_upper, (int64_t)sm_count());
     if (grid <= 0) return cudaSuccess;

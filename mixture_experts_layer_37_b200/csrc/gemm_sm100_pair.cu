@@ -324,13 +324,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 template <int MODE>
 cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                              int64_t rows_cap, cudaStream_t s) {
-    static int max_pairs[64] = {0};
+    static std::atomic<int> max_pairs[64];  // resident clusters per device, 0 until measured
     int dev = 0;
     cudaGetDevice(&dev);
-    int pairs_cap = 0;
-    if (dev < 64 && max_pairs[dev] > 0) {
-        pairs_cap = max_pairs[dev];
-    } else {
+    int pairs_cap = dev < 64 ? max_pairs[dev].load(std::memory_order_acquire) : 0;
+    if (pairs_cap <= 0) {
         cudaError_t err =
             cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemP);
         if (err != cudaSuccess) return err;
@@ -349,7 +347,7 @@ cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const 
         err = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<MODE>, &cfg);
         if (err != cudaSuccess || n <= 0) n = sm_count() / 2;
         pairs_cap = n;
-        if (dev < 64) max_pairs[dev] = n;
+        if (dev < 64) max_pairs[dev].store(n, std::memory_order_release);
     }
     const int64_t tiles_upper = (rows_cap / BMP + p.E) * (int64_t)p.n_tiles;
     const int pairs = (int)min64(tiles_upper, (int64_t)pairs_cap);

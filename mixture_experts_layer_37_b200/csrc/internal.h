@@ -2,6 +2,8 @@
 // translation units.  Internal to libmoe.
 #pragma once
 
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -149,6 +151,18 @@ cudaError_t launch_quantize_int8(const void* w, bool bf16, int64_t E, int64_t K,
 cudaError_t launch_selftest_wait(DevStatus st, cudaStream_t s);
 
 int sm_count();
+
+// Raises a kernel's dynamic shared-memory limit once per device.  Safe from
+// several host threads: concurrent first calls may both set it (idempotent).
+template <class Kernel>
+cudaError_t ensure_smem_attr(std::atomic<bool> (&done)[64], Kernel kernel, int bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    const cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err == cudaSuccess && dev < 64) done[dev].store(true, std::memory_order_release);
+    return err;
+}
 
 // Records `ev` on `s`; while `s` is being captured into a CUDA graph, as an
 // external record, so that the event still marks (and times) each replay.

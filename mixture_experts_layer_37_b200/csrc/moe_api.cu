@@ -10,20 +10,16 @@
 namespace moe {
 
 int sm_count() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];  // per device, 0 until queried
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 64) {
-        int n = 0;
+    int n = dev < 64 ? cached[dev].load(std::memory_order_relaxed) : 0;
+    if (n == 0) {
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        return n > 0 ? n : 1;
+        if (n <= 0) n = 1;
+        if (dev < 64) cached[dev].store(n, std::memory_order_relaxed);
     }
-    if (cached[dev] == 0) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 1;
-    }
-    return cached[dev];
+    return n;
 }
 
 }  // namespace moe

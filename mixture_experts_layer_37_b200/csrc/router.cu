@@ -405,15 +405,9 @@ cudaError_t launch_bf16_tpc(RouterArgs a, cudaStream_t s) {
     a.tpc = TPC;
     const size_t smem = (size_t)union_bytes_for<NT>(a.d) + tail_bytes_for(TPC);
     const size_t smem_max = (size_t)union_bytes_for<NT>(1 << 30) + tail_bytes_for(kMaxTpc);
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(router_bf16_kernel<NT, TPC>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    const cudaError_t err = ensure_smem_attr(attr, router_bf16_kernel<NT, TPC>, (int)smem_max);
+    if (err != cudaSuccess) return err;
     const int grid = (int)((a.T + TPC - 1) / TPC);
     router_bf16_kernel<NT, TPC><<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
@@ -431,14 +425,9 @@ template <int EP>
 cudaError_t launch_f32_ep(RouterArgs a, cudaStream_t s) {
     a.tpc = kChunkTokens;
     const size_t smem = kSlabBytes + tail_bytes_for(a.tpc);
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(router_f32_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    const cudaError_t err = ensure_smem_attr(attr, router_f32_kernel<EP>, (int)smem);
+    if (err != cudaSuccess) return err;
     const int grid = (int)((a.T + a.tpc - 1) / a.tpc);
     router_f32_kernel<EP><<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();

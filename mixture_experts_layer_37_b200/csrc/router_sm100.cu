@@ -306,14 +306,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
 template <int EP>
 cudaError_t launch_ep(const CUtensorMap& mx, const CUtensorMap& mw, const RouterTcArgs& args, cudaStream_t s) {
-    static bool attr[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !attr[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(router_tc_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRSmem);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) attr[dev] = true;
-    }
+    static std::atomic<bool> attr[64];
+    const cudaError_t err = ensure_smem_attr(attr, router_tc_kernel<EP>, kRSmem);
+    if (err != cudaSuccess) return err;
     const int ntiles = (int)((args.r.T + RBM - 1) / RBM);
     const int grid = ntiles < sm_count() ? ntiles : sm_count();
     router_tc_kernel<EP><<<grid, kRThreads, kRSmem, s>>>(mx, mw, args);
