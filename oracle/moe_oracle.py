@@ -51,6 +51,17 @@ DESIGN.md):
       weights, applied to every token (padding included) with weight 1 and
       added after the routed terms: out[t] = sum_j w[t,j] y(t,j) + sum_s y_s(t).
 
+  R19 expert parallelism ([LLaMA4-MoE] §2.5, [MoE-basics] §4.1: each GPU
+      holds some of the experts; tokens go to the GPUs of their experts by an
+      all-to-all and the results come back by a second one): with E experts
+      over `world` ranks, rank o holds the contiguous block
+      [o*E/world, (o+1)*E/world) (the page's example puts 32 experts on 8
+      GPUs, 4 on each).  An owner's receive buffer groups its experts' rows by
+      expert in ascending id, each expert's rows in the batch's token order:
+      the single-device grouping restricted to the owner's experts.  Capacity,
+      drops and statistics are those of the whole batch, so the layer's
+      result does not depend on `world`.
+
 Parity pins: every function here is pinned by tests/test_oracle_pins.py
 (worked example, closed forms, brute force, invariants, library
 cross-checks); none is "parity unpinned".
@@ -378,6 +389,50 @@ def forward(wl, inputs: dict, logits_feed: Optional[np.ndarray] = None,
             xr = to_f64(inputs["x"][toks], wl.dtype)
         out = out + shared_outputs(wl, inputs, xr)
     return {**r, "out": out, "tokens": toks, "y": y}
+
+
+# --------------------------------------------------------------------------
+# expert parallelism
+# --------------------------------------------------------------------------
+def expert_owner(e, E: int, world: int):
+    """Reading R19: the rank holding expert e when E experts are split over
+    `world` ranks in contiguous blocks of E/world ([MoE-basics] §4.1)."""
+    assert world >= 1 and E % world == 0
+    return np.asarray(e) // (E // world)
+
+
+def expert_parallel_layout(idx: np.ndarray, slot: np.ndarray, E: int, world: int) -> dict:
+    """Reading R19: the row each kept assignment takes in the receive buffer of
+    the rank that holds its expert ([LLaMA4-MoE] §2.5; [MoE-basics] §4.1).
+    An owner's rows are grouped by its experts in ascending id, and each
+    expert's rows follow the batch's token order ([LLaMA4-MoE] §2.4 grouping).
+
+    ``idx`` [T,k] are the selected experts (-1 = padding) and ``slot`` [T,k]
+    the single-device dispatch, of which only "kept" (slot >= 0) is read.
+    Returns owner [T,k] and row [T,k] (-1 where dropped), recv_offsets
+    [world, E/world + 1] (each owner's per-expert row offsets) and recv_src, a
+    list over owners of the assignment t*k + j held in each row."""
+    T, k = idx.shape
+    El = E // world
+    flat = idx.reshape(-1).astype(np.int64)
+    kept = slot.reshape(-1) >= 0
+    owner = np.full(T * k, -1, dtype=np.int64)
+    row = np.full(T * k, -1, dtype=np.int64)
+    recv_offsets = np.zeros((world, El + 1), dtype=np.int64)
+    recv_src = []
+    for o in range(world):
+        mine = [e for e in range(E) if int(expert_owner(e, E, world)) == o]
+        rows_o = []
+        for el, e in enumerate(mine):
+            recv_offsets[o, el] = len(rows_o)
+            for a in np.nonzero(kept & (flat == e))[0]:  # ascending assignment = token order
+                owner[a] = o
+                row[a] = len(rows_o)
+                rows_o.append(int(a))
+        recv_offsets[o, len(mine):] = len(rows_o)
+        recv_src.append(np.array(rows_o, dtype=np.int64))
+    return {"owner": owner.reshape(T, k), "row": row.reshape(T, k), "recv_offsets": recv_offsets,
+            "recv_src": recv_src}
 
 
 def shared_outputs(wl, inputs: dict, xr: np.ndarray) -> np.ndarray:

@@ -461,12 +461,86 @@ def check_int8_quantization(o):
     assert np.abs(a["out"] - o.forward(wl.with_(weights="native"), inp)["out"]).max() > 1e-9  # quantisation shows
 
 
+def check_expert_parallel_layout(o):
+    """Reading R19 (expert parallelism, LLaMA4-MoE page §2.5, MoE-basics page
+    §4.1).  Hand cases (E=4 on 2 ranks: experts 0 and 1 on rank 0, 2 and 3 on
+    rank 1; with and without drops); one rank reduces to the single-device
+    dispatch; one expert per rank gives row = slot - offsets[e]; an independent
+    simulation of the all-to-all over random contiguous token slices (each
+    source rank sends every owner its kept rows expert by expert, and the owner
+    stacks each expert's parts in source-rank order) gives the same rows; and
+    the layer computed owner by owner equals the single-device layer."""
+    idx = np.array([[3, 0], [1, 3], [0, 2]], dtype=np.int32)
+    lay = o.expert_parallel_layout(idx, o.dispatch(idx, 4, 3)["slot"], 4, 2)
+    assert lay["owner"].tolist() == [[1, 0], [0, 1], [0, 1]]
+    assert lay["row"].tolist() == [[1, 0], [2, 2], [1, 0]]
+    assert lay["recv_offsets"].tolist() == [[0, 2, 3], [0, 1, 3]]
+    assert [r.tolist() for r in lay["recv_src"]] == [[1, 4, 2], [5, 0, 3]]
+    lay = o.expert_parallel_layout(idx, o.dispatch(idx, 4, 1)["slot"], 4, 2)   # cap 1: assignments 3 and 4 dropped
+    assert lay["owner"].tolist() == [[1, 0], [0, -1], [-1, 1]]
+    assert lay["row"].tolist() == [[1, 0], [1, -1], [-1, 0]]
+    assert lay["recv_offsets"].tolist() == [[0, 1, 2], [0, 1, 2]]
+    rng = np.random.default_rng(19)
+    for trial in range(150):
+        world = int(rng.choice([1, 2, 3, 4]))
+        El = int(rng.integers(1, 4))
+        E = world * El
+        k = int(rng.integers(1, min(E, 3) + 1))
+        T = int(rng.integers(0, 12))
+        idx = o.select_topk(rng.integers(-3, 4, size=(T, E)).astype(np.float64), k)
+        idx[rng.random(T) < 0.15] = -1                     # padding tokens (R16)
+        cap = int(rng.integers(0, T + 2))
+        d = o.dispatch(idx, E, cap)
+        lay = o.expert_parallel_layout(idx, d["slot"], E, world)
+        keep = d["slot"] >= 0
+        assert np.array_equal(lay["row"] >= 0, keep) and np.array_equal(lay["owner"] >= 0, keep)
+        if world == 1:
+            assert np.array_equal(lay["row"], d["slot"])
+            assert lay["recv_offsets"][0].tolist() == d["offsets"].tolist()
+        if El == 1:
+            assert np.array_equal(lay["row"][keep], d["slot"][keep] - d["offsets"][idx[keep]])
+        cuts = sorted(int(c) for c in rng.integers(0, T + 1, size=world - 1))
+        bounds = [0, *cuts, T]
+        part = {}
+        for src in range(world):
+            for own in range(world):
+                for e in range(own * El, (own + 1) * El):
+                    part.setdefault((own, e), []).extend(
+                        t * k + j for t in range(bounds[src], bounds[src + 1]) for j in range(k)
+                        if idx[t, j] == e and d["slot"][t, j] >= 0)
+        for own in range(world):
+            rows = [a for e in range(own * El, (own + 1) * El) for a in part[(own, e)]]
+            assert lay["recv_src"][own].tolist() == rows
+            sizes = [len(part[(own, e)]) for e in range(own * El, (own + 1) * El)]
+            assert lay["recv_offsets"][own].tolist() == [0, *np.cumsum(sizes).tolist()]
+            for r_, a in enumerate(rows):
+                assert lay["owner"].reshape(-1)[a] == own and lay["row"].reshape(-1)[a] == r_
+    # the layer, computed owner by owner on the received rows, equals the single-device layer
+    wl = _wl(T=29, d=8, ffn=12, E=6, k=2, capacity_factor=0.8, seed=12, w_std=0.3)
+    inp = W.make_inputs(wl)
+    x = o.to_f64(inp["x"], wl.dtype)
+    ref = o.forward(wl, inp)
+    lay = o.expert_parallel_layout(ref["idx"], ref["slot"], wl.E, 3)
+    y = {}
+    for own in range(3):
+        src = lay["recv_src"][own]
+        offs = lay["recv_offsets"][own]
+        for el in range(2):
+            rows = src[offs[el]:offs[el + 1]]
+            if rows.size:
+                ye = o.expert_apply(wl, o.expert_weights_f64(wl, inp, own * 2 + el), x[rows // wl.k])
+                y.update({int(a): ye[i] for i, a in enumerate(rows)})
+    out = o.combine(y, ref["slot"], ref["w"], wl.T, wl.d)
+    assert (ref["slot"] < 0).any(), "the case must exercise drops"
+    np.testing.assert_allclose(out, ref["out"], rtol=1e-12, atol=1e-14)
+
+
 CHECKS = [check_worked_example, check_uniform_alpha, check_sums_to_one, check_topk_bruteforce,
           check_tie_lower_id, check_renorm_is_selected_softmax, check_softmax_closed_form,
           check_capacity, check_dispatch_hand_case, check_dispatch_bruteforce,
           check_activation_closed_forms, check_dense_reduction, check_teaching_layer,
           check_combine_properties, check_drop_path_end_to_end, check_empty, check_padding_mask,
-          check_shared_experts, check_int8_quantization]
+          check_shared_experts, check_int8_quantization, check_expert_parallel_layout]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
@@ -586,7 +660,34 @@ def _quant_truncating(w):
     return q, s
 
 
+def _ep_owner_round_robin(e, E, world):
+    return np.asarray(e) % world
+
+
+def _ep_layout_token_major(idx, slot, E, world):
+    # an owner's rows in token order across its experts (not grouped by expert)
+    T, k = idx.shape
+    El = E // world
+    flat = idx.reshape(-1).astype(np.int64)
+    kept = slot.reshape(-1) >= 0
+    owner = np.full(T * k, -1, dtype=np.int64)
+    row = np.full(T * k, -1, dtype=np.int64)
+    recv_offsets = np.zeros((world, El + 1), dtype=np.int64)
+    recv_src = []
+    for own in range(world):
+        rows = [int(a) for a in np.nonzero(kept & (flat >= 0) & (flat // El == own))[0]]
+        for r_, a in enumerate(rows):
+            owner[a], row[a] = own, r_
+        for el in range(El + 1):
+            recv_offsets[own, el] = sum(1 for a in rows if flat[a] - own * El < el)
+        recv_src.append(np.array(rows, dtype=np.int64))
+    return {"owner": owner.reshape(T, k), "row": row.reshape(T, k), "recv_offsets": recv_offsets,
+            "recv_src": recv_src}
+
+
 MUTANTS = {
+    "ep_owner_round_robin": dict(expert_owner=_ep_owner_round_robin),
+    "ep_rows_token_major": dict(expert_parallel_layout=_ep_layout_token_major),
     "int8_global_scale": dict(quantize_int8=_quant_global_scale),
     "int8_truncating_codes": dict(quantize_int8=_quant_truncating),
     "padding_selects_experts": dict(mask_padding=_mask_ignored),
