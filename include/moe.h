@@ -61,7 +61,9 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,  /* valid shape this build does not run (e.g. E > 64) */
     MOE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moe_workspace_size */
     MOE_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
-    MOE_ERR_TIMEOUT = 5       /* a bounded device wait gave up (see moe_check_device_status) */
+    MOE_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (see moe_check_device_status) */
+    MOE_ERR_RANGE = 6         /* a device-side bounds check refused a row (inconsistent counts;
+                                 see moe_check_device_status and the expert-parallel calls) */
 } moe_status_t;
 
 typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype_t;
@@ -314,6 +316,89 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
                            const void* x, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
                            cudaStream_t stream);
 
+/* ---- Expert parallelism: experts sharded over ranks --------------------
+ * "Hand-building a LLaMA4-MoE" §2.5 and the MoE-basics page §4.1: each GPU
+ * holds some of the experts; an all-to-all sends every token to the GPUs
+ * holding its experts and a second one brings the results back.  Here `world`
+ * ranks (1..8, the GPUs of one NVSwitch node) each hold
+ *   - a contiguous slice of one batch of T_global tokens (cfg->T tokens,
+ *     slices in rank order), as in the data-parallel calls above, and
+ *   - the experts [rank*E/world, (rank+1)*E/world) (E % world == 0), whose
+ *     weights are passed as a pool of E/world experts ([E/world, d, ffn] ...);
+ *     the router weights and the shared experts are replicated.
+ * Capacity, drops and statistics are the whole batch's; every expert's rows
+ * reach its rank in the batch's token order, so the layer output equals one
+ * moe_forward over the whole batch, bit for bit.
+ *
+ * Each rank owns two receive buffers of moe_ep_recv_rows rows: x_recv
+ * [rows, d] and y_recv [rows, d] (config dtype), on its own GPU.  The
+ * dispatch and combine calls take the array of every rank's buffer
+ * (x_recv[r] / y_recv[r], r = 0..world-1, HOST array of DEVICE pointers that
+ * this rank can dereference: its own buffer and its peers' buffers mapped
+ * into this process, e.g. with moe_ipc_open over NVLink).  The kernels
+ * store token rows straight into the owners' x_recv (dispatch) and load
+ * expert rows straight from the owners' y_recv (combine): the two
+ * all-to-alls are fused into the scatter and the weighted sum.
+ *
+ * Sequence on every rank (the same steps on all ranks, even with no rows):
+ *   1. moe_ep_route: router and top-k of the slice, local_counts [E] int32
+ *      and local_psum [E] float64 (device).
+ *   2. all-gather local_counts / local_psum in rank order into all_counts
+ *      [world, E] / all_psum [world, E] (e.g. NCCL).
+ *   3. moe_ep_dispatch: capacity left, rows into the owners' x_recv,
+ *      outputs->slot [T,k] = row in the owner's y_recv (or -1), recv_offsets
+ *      [E/world + 1] = this rank's received rows per local expert, and the
+ *      whole batch's counts, offsets (single-device layout), f, p, l_aux.
+ *   4. barrier: every rank's step 3 finished (e.g. a one-word NCCL
+ *      all-reduce on the stream).
+ *   5. moe_ep_expert_ffn: grouped GEMMs over x_recv -> y_recv with this
+ *      rank's experts; the shared experts over the slice's tokens.
+ *   6. barrier: every rank's step 5 finished.
+ *   7. moe_ep_combine: outputs->out [T,d] of the slice.
+ * The receive buffers must not be reused by the next forward's step 3 before
+ * every rank's step 7 finished (the all-gather of step 2 orders that).
+ * All four calls use one workspace of moe_ep_workspace_size bytes per rank.
+ * The padding mask is not supported here. */
+moe_status_t moe_ep_recv_rows(const moe_config_t* cfg, int64_t T_global, int32_t world, int64_t* rows);
+moe_status_t moe_ep_workspace_size(const moe_config_t* cfg, int64_t T_global, int32_t world, size_t* bytes);
+moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t world, const moe_weights_t* weights,
+                          const void* x, const float* logits_in, moe_outputs_t* outputs, int32_t* local_counts,
+                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream);
+/* all_counts / all_psum: DEVICE [world, E] as gathered in step 2; counts that
+ * do not match the routing make the kernels refuse rows (MOE_ERR_RANGE from
+ * moe_check_device_status; memory stays in bounds). */
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
+                             const double* all_psum, int32_t world, int32_t rank, const void* x,
+                             void* const* x_recv, moe_outputs_t* outputs, int32_t* recv_offsets, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+/* weights: the E/world local experts (and the shared experts); x: the
+ * slice's tokens (read only by the shared experts; may be NULL without
+ * them); x_recv / y_recv / recv_offsets: this rank's own. */
+moe_status_t moe_ep_expert_ffn(const moe_config_t* cfg, int64_t T_global, int32_t world,
+                               const moe_weights_t* weights, const void* x, const void* x_recv,
+                               const int32_t* recv_offsets, void* y_recv, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+moe_status_t moe_ep_combine(const moe_config_t* cfg, int64_t T_global, int32_t world, const void* const* y_recv,
+                            moe_outputs_t* outputs, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ---- Device buffers shared between processes (CUDA IPC) ----------------
+ * A record that names a device buffer for other processes of the node.
+ * moe_ipc_export fills it for the buffer at dev_ptr (inside any cudaMalloc
+ * allocation: the record holds the allocation's handle and dev_ptr's offset
+ * in it); moe_ipc_open maps it into the calling process (with peer access
+ * enabled, so that kernels load and store it over NVLink) and returns the
+ * device pointer of dev_ptr there; moe_ipc_close unmaps it.  The exporting
+ * process keeps the allocation alive until every importer has closed it.
+ * A process cannot open its own records.  MOE_ERR_CUDA when CUDA refuses. */
+typedef struct {
+    uint8_t handle[64];   /* cudaIpcMemHandle_t of the allocation */
+    uint64_t offset;      /* dev_ptr - allocation base */
+    uint64_t bytes;       /* allocation size - offset */
+} moe_ipc_buffer_t;
+moe_status_t moe_ipc_export(const void* dev_ptr, moe_ipc_buffer_t* record);
+moe_status_t moe_ipc_open(const moe_ipc_buffer_t* record, void** dev_ptr);
+moe_status_t moe_ipc_close(void* dev_ptr, const moe_ipc_buffer_t* record);
+
 /* moe_forward, recording stage_events[i] on `stream` just before kernel
  * launch i and stage_events[n] after the last launch, n =
  * moe_forward_launch_count(cfg) (stage_events: caller-created CUDA events,
@@ -344,7 +429,9 @@ moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* we
 /* Synchronises `stream`, then reads and clears the workspace status word.
  * Returns MOE_ERR_TIMEOUT if a bounded device wait gave up since the last
  * check (`*site`, if not NULL, receives the code of the first wait that gave
- * up), MOE_ERR_CUDA if the synchronisation failed, else MOE_OK. */
+ * up), else MOE_ERR_RANGE if a device-side bounds check refused a row (the
+ * expert-parallel calls given counts that do not match the routing),
+ * MOE_ERR_CUDA if the synchronisation failed, else MOE_OK. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t* site);
 
 /* ---- Pipelined forwards on host-resident batches ------------------------

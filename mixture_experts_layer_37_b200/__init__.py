@@ -21,7 +21,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+(MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
+ MOE_ERR_RANGE) = range(7)
+MOE_MAX_RANKS = 8  # ranks of one expert-parallel group
 MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_ACT_SWIGLU, MOE_ACT_GELU_BIAS = 0, 1
 MOE_ROUTER_AUTO, MOE_ROUTER_WARP_MMA, MOE_ROUTER_TCGEN05 = 0, 1, 2
@@ -110,7 +112,9 @@ EXPORTED_SYMBOLS = ("moe_status_string", "moe_capacity", "moe_max_rows", "moe_wo
                     "moe_selftest_bounded_wait", "moe_forward_launch_count", "moe_forward_profiled",
                     "moe_dispatch_noalloc", "moe_dp_workspace_size", "moe_dp_max_rows", "moe_dp_route",
                     "moe_dp_finish", "moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_wait",
-                    "moe_pipeline_check", "moe_pipeline_destroy", "moe_quantize_int8")
+                    "moe_pipeline_check", "moe_pipeline_destroy", "moe_quantize_int8", "moe_ep_recv_rows",
+                    "moe_ep_workspace_size", "moe_ep_route", "moe_ep_dispatch", "moe_ep_expert_ffn",
+                    "moe_ep_combine", "moe_ipc_export", "moe_ipc_open", "moe_ipc_close")
 
 
 # ---------------------------------------------------------------- config
@@ -425,6 +429,121 @@ def moe_dp_finish(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: in
     oc = _outputs_c(outputs)
     _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank),
              ctypes.byref(wc), _ptr(x), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_finish")
+
+
+# ---------------------------------------------------------------- expert parallelism
+_EXPERT_KEYS = ("w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2", "w_gate_scale", "w_up_scale", "w_down_scale",
+                "w1_scale", "w2_scale")
+
+
+def local_expert_weights(weights: dict, world: int, rank: int) -> dict:
+    """The weights rank `rank` holds under expert parallelism: its contiguous
+    block of E/world routed experts (views along the expert axis), with the
+    router and the shared experts as they are (replicated)."""
+    out = dict(weights)
+    for n in _EXPERT_KEYS:
+        if n in weights and weights[n] is not None:
+            E = weights[n].shape[0]
+            el = E // world
+            out[n] = weights[n][rank * el:(rank + 1) * el]
+    return out
+
+
+def _ptr_array(ptrs) -> ctypes.Array:
+    vals = [p.data_ptr() if isinstance(p, torch.Tensor) else int(p) for p in ptrs]
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def _ep_fn(name: str, argtypes: list):
+    f = getattr(lib(), name)
+    f.argtypes = argtypes
+    f.restype = ctypes.c_int
+    return f
+
+
+def moe_ep_recv_rows(cfg: MoEConfig, T_global: int, world: int) -> int:
+    v = ctypes.c_int64()
+    f = _ep_fn("moe_ep_recv_rows", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64)])
+    _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), ctypes.byref(v)), "moe_ep_recv_rows")
+    return v.value
+
+
+def moe_ep_workspace_size(cfg: MoEConfig, T_global: int, world: int) -> int:
+    v = ctypes.c_size_t()
+    f = _ep_fn("moe_ep_workspace_size", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)])
+    _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), ctypes.byref(v)), "moe_ep_workspace_size")
+    return v.value
+
+
+def moe_ep_route(cfg: MoEConfig, T_global: int, world: int, weights: dict, x, outputs: dict, local_counts,
+                 local_psum, ws: Workspace, logits_in=None, stream=None) -> None:
+    f = _ep_fn("moe_ep_route", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P, _P,
+                                ctypes.POINTER(MoEOutputsC), _P, _P, _P, ctypes.c_size_t, _P])
+    wc = _weights_c(weights)
+    oc = _outputs_c(outputs)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), ctypes.byref(wc), _ptr(x), _ptr(logits_in),
+             ctypes.byref(oc), _ptr(local_counts), _ptr(local_psum), ws.ptr, ws.nbytes, _stream(stream)),
+           "moe_ep_route")
+
+
+def moe_ep_dispatch(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: int, rank: int, x, x_recv,
+                    outputs: dict, recv_offsets, ws: Workspace, stream=None) -> None:
+    """x_recv: every rank's receive buffer (tensors on this device, or device
+    pointers this process can dereference), in rank order."""
+    f = _ep_fn("moe_ep_dispatch", [_CFG, ctypes.c_int64, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                   ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(MoEOutputsC), _P, _P,
+                                   ctypes.c_size_t, _P])
+    oc = _outputs_c(outputs)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank), _ptr(x),
+             _ptr_array(x_recv), ctypes.byref(oc), _ptr(recv_offsets), ws.ptr, ws.nbytes, _stream(stream)),
+           "moe_ep_dispatch")
+
+
+def moe_ep_expert_ffn(cfg: MoEConfig, T_global: int, world: int, weights: dict, x, x_recv, recv_offsets, y_recv,
+                      ws: Workspace, stream=None) -> None:
+    """weights: this rank's experts (local_expert_weights) and the shared experts."""
+    f = _ep_fn("moe_ep_expert_ffn", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P, _P, _P,
+                                     _P, _P, ctypes.c_size_t, _P])
+    wc = _weights_c(weights)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), ctypes.byref(wc), _ptr(x), _ptr(x_recv),
+             _ptr(recv_offsets), _ptr(y_recv), ws.ptr, ws.nbytes, _stream(stream)), "moe_ep_expert_ffn")
+
+
+def moe_ep_combine(cfg: MoEConfig, T_global: int, world: int, y_recv, outputs: dict, ws: Workspace,
+                   stream=None) -> None:
+    """y_recv: every rank's output buffer, in rank order (as x_recv of moe_ep_dispatch)."""
+    f = _ep_fn("moe_ep_combine", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
+                                  ctypes.POINTER(MoEOutputsC), _P, ctypes.c_size_t, _P])
+    oc = _outputs_c(outputs)
+    _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), _ptr_array(y_recv), ctypes.byref(oc), ws.ptr,
+             ws.nbytes, _stream(stream)), "moe_ep_combine")
+
+
+class MoEIpcBufferC(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_uint8 * 64), ("offset", ctypes.c_uint64), ("bytes", ctypes.c_uint64)]
+
+
+def moe_ipc_export(t: torch.Tensor) -> bytes:
+    """The record (bytes) naming device tensor t's memory for other processes."""
+    rec = MoEIpcBufferC()
+    f = _ep_fn("moe_ipc_export", [_P, ctypes.POINTER(MoEIpcBufferC)])
+    _check(f(t.data_ptr(), ctypes.byref(rec)), "moe_ipc_export")
+    return bytes(rec)
+
+
+def moe_ipc_open(record: bytes) -> int:
+    """Maps another process's exported buffer; returns its device pointer here."""
+    rec = MoEIpcBufferC.from_buffer_copy(record)
+    ptr = ctypes.c_void_p()
+    f = _ep_fn("moe_ipc_open", [ctypes.POINTER(MoEIpcBufferC), ctypes.POINTER(ctypes.c_void_p)])
+    _check(f(ctypes.byref(rec), ctypes.byref(ptr)), "moe_ipc_open")
+    return int(ptr.value)
+
+
+def moe_ipc_close(ptr: int, record: bytes) -> None:
+    rec = MoEIpcBufferC.from_buffer_copy(record)
+    f = _ep_fn("moe_ipc_close", [_P, ctypes.POINTER(MoEIpcBufferC)])
+    _check(f(ptr, ctypes.byref(rec)), "moe_ipc_close")
 
 
 # ---------------------------------------------------------------- pipelined forwards on host batches

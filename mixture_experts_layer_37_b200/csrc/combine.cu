@@ -16,7 +16,10 @@
 namespace moe {
 namespace {
 
-template <bool BF16>
+// EP: the expert rows are read from the output buffer of the rank holding
+// each expert (peer memory over NVLink), so the gather back to token order is
+// this step's all-to-all, fused with the weighted sum.
+template <bool BF16, bool EP>
 __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
     constexpr int U = 4;               // 16-byte vectors per lane per expert row (x2 rows in flight)
     constexpr int VEC = BF16 ? 8 : 4;  // elements per 16-byte vector
@@ -30,16 +33,32 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
     for (int64_t t = warp_g; t < a.T; t += nwarps) {
         int s_l = -1;
         float w_l = 0.f;
+        const uint4* y_l = Y;
         if (lane < a.k) {
             s_l = a.slot[t * a.k + lane];
             w_l = a.topk_w[t * a.k + lane];
+            if constexpr (EP) {
+                if (s_l >= 0) {
+                    const int e = a.topk_idx[t * a.k + lane];
+                    const int r = e >= 0 ? e / a.e_per_rank : kMaxRanks;
+                    y_l = r < kMaxRanks ? static_cast<const uint4*>(a.y_src[r]) : nullptr;
+                    if (y_l == nullptr || s_l >= a.row_limit) {
+                        report_range(a.st, SITE_EP_COMBINE_ROW);
+                        s_l = -1;
+                    }
+                }
+            }
         }
         int sj[kMaxTopK];
         float wj[kMaxTopK];
+        const uint4* yj[EP ? kMaxTopK : 1];
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) {
             sj[j] = __shfl_sync(0xffffffffu, s_l, j);
             wj[j] = __shfl_sync(0xffffffffu, w_l, j);
+            if constexpr (EP)
+                yj[j] = reinterpret_cast<const uint4*>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(y_l), j));
         }
         for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
             float acc[U][VEC];
@@ -51,12 +70,18 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
             for (int j = 0; j < a.k; j += 2) {
                 const int s0 = sj[j];
                 const int s1 = (j + 1 < a.k) ? sj[j + 1] : -1;
+                const uint4* Y0 = Y;
+                const uint4* Y1 = Y;
+                if constexpr (EP) {
+                    Y0 = yj[j];
+                    Y1 = (j + 1 < a.k) ? yj[j + 1] : Y;
+                }
                 uint4 y0[U], y1[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const bool in = v0 + 32 * u < nvec;
-                    if (in && s0 >= 0) y0[u] = Y[(int64_t)s0 * nvec + v0 + 32 * u];
-                    if (in && s1 >= 0) y1[u] = Y[(int64_t)s1 * nvec + v0 + 32 * u];
+                    if (in && s0 >= 0) y0[u] = Y0[(int64_t)s0 * nvec + v0 + 32 * u];
+                    if (in && s1 >= 0) y1[u] = Y1[(int64_t)s1 * nvec + v0 + 32 * u];
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -185,10 +210,15 @@ __global__ void selftest_wait_kernel(DevStatus st) {
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const int64_t blocks = min64((a.T + 7) / 8, (int64_t)sm_count() * 8);
-    if (bf16)
-        combine_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(a);
+    const bool ep = a.e_per_rank > 0;
+    if (bf16 && ep)
+        combine_kernel<true, true><<<(unsigned)blocks, 256, 0, s>>>(a);
+    else if (bf16)
+        combine_kernel<true, false><<<(unsigned)blocks, 256, 0, s>>>(a);
+    else if (ep)
+        combine_kernel<false, true><<<(unsigned)blocks, 256, 0, s>>>(a);
     else
-        combine_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(a);
+        combine_kernel<false, false><<<(unsigned)blocks, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

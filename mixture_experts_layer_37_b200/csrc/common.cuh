@@ -21,6 +21,9 @@ constexpr int kMaxTopK = 8;
 // resets the counter to 0, and moe_workspace_init zeroes it).
 constexpr int kStatusCounterWord = 4;
 constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrRange = 2u;  // a row index failed a bounds check; the access was skipped
+// Ranks of one expert-parallel group (the GPUs of one NVSwitch node).
+constexpr int kMaxRanks = 8;
 enum WaitSite : uint32_t {
     SITE_NONE = 0,
     SITE_GEMM_PRODUCER_EMPTY = 0x101,
@@ -31,6 +34,9 @@ enum WaitSite : uint32_t {
     SITE_GEMM_PRODUCER_DRAIN = 0x106,
     SITE_SELFTEST_MBAR = 0x201,
     SITE_SELFTEST_FLAG = 0x202,
+    SITE_EP_SCATTER_ROW = 0x301,
+    SITE_EP_PREPARE_ROWS = 0x302,
+    SITE_EP_COMBINE_ROW = 0x303,
 };
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -48,6 +54,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void report_timeout(const DevStatus& st, uint32_t site) {
     atomicOr(st.word, kErrTimeout);
+    atomicCAS(st.word + 1, 0u, site);
+}
+
+__device__ __forceinline__ void report_range(const DevStatus& st, uint32_t site) {
+    atomicOr(st.word, kErrRange);
     atomicCAS(st.word + 1, 0u, site);
 }
 

@@ -45,10 +45,12 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
 
 // One CTA per chunk of kChunkTokens tokens (<= 256 assignments): ranks,
 // capacity test, slot and src_assign, then the row copies x[t] -> x_perm[slot]
-// (each warp copies two rows at a time with 16-byte vectors).
+// (each warp copies two rows at a time with 16-byte vectors).  Under expert
+// parallelism the destination is the receive buffer of the expert's rank, so
+// the copies are this step's all-to-all: stores into peer memory over NVLink.
 __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a) {
     __shared__ int sWarpBase[kScatterWarps][kMaxExperts];
-    __shared__ int sSlot[kScatterThreads];
+    __shared__ uint4* sDst[kScatterThreads];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, k = a.k;
     const int chunk = blockIdx.x;
@@ -82,22 +84,32 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
         const int cap = a.cap_e != nullptr ? a.cap_e[e] : a.cap;
         if (rank < cap) {
             s = a.offsets[e] + rank;
-            a.src_assign[s] = (int32_t)(a_base + tid);
+            if (a.row_limit > 0 && (s < 0 || s >= a.row_limit)) {
+                if (a.st.word != nullptr) report_range(a.st, SITE_EP_SCATTER_ROW);
+                s = -1;
+            } else if (a.src_assign != nullptr) {
+                a.src_assign[s] = (int32_t)(a_base + tid);
+            }
         }
     }
     if (tid < nA) a.slot[a_base + tid] = s;
-    if (a.x_perm == nullptr) return;  // rows gathered by the first GEMM instead
-    sSlot[tid] = s;
+    const bool ep = a.e_per_rank > 0;
+    if (a.x_perm == nullptr && !ep) return;  // rows gathered by the first GEMM instead
+    uint4* dst = nullptr;
+    if (s >= 0) {
+        void* base = ep ? a.x_dst[e / a.e_per_rank] : a.x_perm;
+        dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(base) + (int64_t)s * a.row_bytes);
+    }
+    sDst[tid] = dst;
     __syncthreads();
     // row gather: each warp copies two rows at a time (16-byte vectors, up to
     // 16 loads in flight per lane); dropped assignments copy nothing
     const int vecs = a.row_bytes / 16;
     const uint4* X = static_cast<const uint4*>(a.x);
-    uint4* XP = static_cast<uint4*>(a.x_perm);
     for (int q = warp; q < nA; q += 2 * kScatterWarps) {
         const int q1 = q + kScatterWarps;
-        const int s0 = sSlot[q];
-        const int s1 = q1 < nA ? sSlot[q1] : -1;
+        uint4* d0 = sDst[q];
+        uint4* d1 = q1 < nA ? sDst[q1] : nullptr;
         const uint4* src0 = X + ((a_base + q) / k) * vecs;
         const uint4* src1 = X + ((a_base + (q1 < nA ? q1 : q)) / k) * vecs;
         for (int v0 = lane; v0 < vecs; v0 += 32 * 8) {
@@ -106,16 +118,16 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
             for (int u = 0; u < 8; ++u) {
                 const int v = v0 + 32 * u;
                 if (v < vecs) {
-                    if (s0 >= 0) b0[u] = src0[v];
-                    if (s1 >= 0) b1[u] = src1[v];
+                    if (d0 != nullptr) b0[u] = src0[v];
+                    if (d1 != nullptr) b1[u] = src1[v];
                 }
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int v = v0 + 32 * u;
                 if (v < vecs) {
-                    if (s0 >= 0) XP[(int64_t)s0 * vecs + v] = b0[u];
-                    if (s1 >= 0) XP[(int64_t)s1 * vecs + v] = b1[u];
+                    if (d0 != nullptr) d0[v] = b0[u];
+                    if (d1 != nullptr) d1[v] = b1[u];
                 }
             }
         }
@@ -170,7 +182,90 @@ __global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
     }
 }
 
+// One CTA: expert-parallel shard preparation (see EpPrepareArgs).  Ranks
+// before this one keep min(base_e, cap) rows of expert e, so this slice's
+// kept rows of e start there within e's block in its owner's buffer; an
+// owner's blocks follow its experts in ascending id, each of size
+// min(total_e, cap), so every expert's rows sit in the batch's token order.
+// The capacity left for this slice is also capped by the slice's own
+// gathered count, so that a slice can never write past its part of e's block.
+// If the gathered counts are negative or would overflow any owner's receive
+// buffer, nothing is kept (cap_e = 0, all offsets 0) and kErrRange is set.
+__global__ void __launch_bounds__(64) ep_prepare_kernel(EpPrepareArgs a) {
+    __shared__ int64_t sBefore[kMaxExperts];
+    __shared__ int64_t sTotal[kMaxExperts];
+    __shared__ int64_t sMine[kMaxExperts];
+    __shared__ double sP[kMaxExperts];
+    __shared__ int sBad;
+    const int e = threadIdx.x;
+    if (e == 0) sBad = 0;
+    __syncthreads();
+    if (e < a.E) {
+        int64_t base = 0, total = 0;
+        double ps = 0.0;
+        for (int r = 0; r < a.world; ++r) {
+            const int c = a.all_counts[(int64_t)r * a.E + e];
+            if (c < 0) sBad = 1;
+            if (r < a.rank) base += c;
+            total += c;
+            ps += a.all_psum[(int64_t)r * a.E + e];
+        }
+        sBefore[e] = base;
+        sTotal[e] = total;
+        sMine[e] = a.all_counts[(int64_t)a.rank * a.E + e];
+        sP[e] = a.T_global > 0 ? ps / (double)a.T_global : 0.0;
+    }
+    __syncthreads();
+    if (e == 0) {
+        for (int o = 0; o < a.world; ++o) {
+            int64_t rows = 0;
+            for (int el = 0; el < a.e_per_rank; ++el) rows += min64(sTotal[o * a.e_per_rank + el], a.cap);
+            if (rows > a.recv_rows) sBad = 1;
+        }
+        if (sBad) report_range(a.st, SITE_EP_PREPARE_ROWS);
+    }
+    __syncthreads();
+    const bool ok = sBad == 0;
+    if (e < a.E) {
+        const int64_t left = min64(a.cap - sBefore[e], sMine[e]);
+        a.cap_e[e] = ok && left > 0 ? (int32_t)left : 0;
+    }
+    if (e == 0) {
+        int64_t off = 0, owner_off = 0;
+        double l = 0.0;
+        for (int i = 0; i < a.E; ++i) {
+            const int el = i % a.e_per_rank;
+            const bool mine = i / a.e_per_rank == a.rank;
+            if (el == 0) owner_off = 0;
+            const int64_t kept = ok ? min64(sTotal[i], a.cap) : 0;
+            a.dest_off[i] = (int32_t)(owner_off + (ok ? min64(sBefore[i], a.cap) : 0));
+            if (mine) a.recv_offsets[el] = (int32_t)owner_off;
+            owner_off += kept;
+            if (mine && el == a.e_per_rank - 1) a.recv_offsets[a.e_per_rank] = (int32_t)owner_off;
+            a.offsets[i] = (int32_t)off;
+            off += kept;
+            const int32_t cnt = ok ? (int32_t)sTotal[i] : 0;
+            a.counts[i] = cnt;
+            const double f = a.T_global > 0 ? (double)cnt / ((double)a.T_global * a.k) : 0.0;
+            a.f[i] = (float)f;
+            a.p[i] = (float)sP[i];
+            l += f * sP[i];
+        }
+        a.offsets[a.E] = (int32_t)off;
+        a.l_aux[0] = (float)((double)a.alpha * a.E * l);
+        if (a.shared_off != nullptr) {
+            a.shared_off[0] = 0;
+            a.shared_off[1] = (int32_t)a.T_local;
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_ep_prepare(const EpPrepareArgs& a, cudaStream_t s) {
+    ep_prepare_kernel<<<1, 64, 0, s>>>(a);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s) {
     dp_prepare_kernel<<<1, 64, 0, s>>>(a);

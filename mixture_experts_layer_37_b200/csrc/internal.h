@@ -73,6 +73,14 @@ struct ScatterArgs {
     int64_t T = 0;
     int E = 0, k = 0, cap = 0, nchunk = 0;
     int row_bytes = 0;              // d * element size (multiple of 16)
+    // expert parallelism (e_per_rank > 0): the rows of expert e go to
+    // x_dst[e / e_per_rank] (the receive buffer of the rank holding e, possibly
+    // a peer's memory), slot = row there; rows at or past row_limit are refused
+    // (slot -1, kErrRange in st); src_assign may be null
+    void* x_dst[kMaxRanks] = {};
+    int e_per_rank = 0;
+    int64_t row_limit = 0;          // > 0: bound of every destination row
+    DevStatus st;
 };
 cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
 
@@ -96,6 +104,32 @@ struct DpPrepareArgs {
 };
 cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s);
 
+// Expert-parallel shard: rank `rank` holds the tokens of its slice and the
+// experts [rank*e_per_rank, (rank+1)*e_per_rank).  From every rank's counts
+// and probability sums ([world, E], gathered in rank order): the capacity
+// left for this slice, the first row in its owner's receive buffer of this
+// slice's kept rows of each expert, this rank's receive offsets as an owner,
+// and the whole batch's counts, offsets, f, p, L_aux.
+struct EpPrepareArgs {
+    const int32_t* all_counts = nullptr;  // [world, E]
+    const double* all_psum = nullptr;     // [world, E]
+    int world = 0, rank = 0, E = 0, e_per_rank = 0, k = 0, cap = 0;
+    int64_t T_global = 0, T_local = 0;
+    int64_t recv_rows = 0;                // rows of every receive buffer
+    float alpha = 0;
+    int32_t* cap_e = nullptr;             // [E] out
+    int32_t* dest_off = nullptr;          // [E] out: row in owner(e)'s buffer of this slice's first kept row of e
+    int32_t* recv_offsets = nullptr;      // [e_per_rank + 1] out: this rank's received rows per local expert
+    int32_t* offsets = nullptr;           // [E+1] out: the whole batch's kept-row offsets (single-device layout)
+    int32_t* counts = nullptr;            // [E] out (global)
+    float* f = nullptr;                   // [E] out
+    float* p = nullptr;                   // [E] out
+    float* l_aux = nullptr;               // [1] out
+    int32_t* shared_off = nullptr;        // [2] out or null: {0, T_local}
+    DevStatus st;
+};
+cudaError_t launch_ep_prepare(const EpPrepareArgs& a, cudaStream_t s);
+
 struct CombineArgs {
     const void* y_perm = nullptr;    // [R_max, d]
     const int32_t* slot = nullptr;   // [T, k]
@@ -105,6 +139,14 @@ struct CombineArgs {
     int n_shared = 0;
     int64_t T = 0;
     int d = 0, k = 0;
+    // expert parallelism (e_per_rank > 0): row slot[t,j] of y_src[topk_idx[t,j] / e_per_rank]
+    // (the output buffer of the rank holding the expert, possibly a peer's memory); slots at or
+    // past row_limit are refused (kErrRange in st)
+    const void* y_src[kMaxRanks] = {};
+    const int32_t* topk_idx = nullptr;
+    int e_per_rank = 0;
+    int64_t row_limit = 0;
+    DevStatus st;
 };
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s);
 cudaError_t launch_aux_from_probs(const int32_t* counts, const float* probs, float* f, float* p, float* l_aux,

@@ -86,10 +86,12 @@ int64_t max_rows(const moe_config_t* c) {
 struct Plan {
     int nchunk;
     int64_t rows;
-    size_t hist, psum, base, cap_e, nreal, shared_off, xperm, h, yperm, hs, ys, total;
+    size_t hist, psum, base, cap_e, nreal, shared_off, ep_dest, xperm, h, yperm, hs, ys, total;
 };
 
-Plan plan_rows(const moe_config_t* c, int64_t rows) {
+// perm_buffers = false: no x_perm / y_perm (the expert-parallel calls use the
+// caller's receive buffers instead).
+Plan plan_rows(const moe_config_t* c, int64_t rows, bool perm_buffers = true) {
     Plan p;
     p.nchunk = (int)((c->T + kChunkTokens - 1) / kChunkTokens);
     p.rows = rows;
@@ -108,12 +110,15 @@ Plan plan_rows(const moe_config_t* c, int64_t rows) {
     off = align_up(off + (size_t)p.nchunk * 4, 1024);
     p.shared_off = off;
     off = align_up(off + 2 * 4, 1024);
+    p.ep_dest = off;
+    off = align_up(off + E * 4, 1024);
+    const size_t perm_rows = perm_buffers ? (size_t)p.rows : 0;
     p.xperm = off;
-    off = align_up(off + (size_t)p.rows * c->d * s, 1024);
+    off = align_up(off + perm_rows * c->d * s, 1024);
     p.h = off;
     off = align_up(off + (size_t)p.rows * c->ffn * s, 1024);
     p.yperm = off;
-    off = align_up(off + (size_t)p.rows * c->d * s, 1024);
+    off = align_up(off + perm_rows * c->d * s, 1024);
     // shared experts: one [T, ffn] intermediate reused in turn, and each one's [T, d] output
     p.hs = off;
     off = align_up(off + (c->n_shared > 0 ? (size_t)c->T * c->ffn * s : 0), 1024);
@@ -143,6 +148,24 @@ moe_status_t check_dp(const moe_config_t* c, int64_t T_global) {
     if (T_global < c->T) return MOE_ERR_INVALID_ARG;
     if (T_global * (int64_t)c->k >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
+}
+
+// Expert-parallel shard over `world` ranks: rows of every receive buffer
+// (the most rows E/world experts can keep of the whole batch).
+int64_t ep_recv_rows(const moe_config_t* c, int64_t T_global, int world) {
+    const int64_t cap = dp_cap_used(c, T_global);
+    const int64_t a = T_global * c->k, b = (int64_t)(c->E / world) * cap;
+    return a < b ? a : b;
+}
+moe_status_t check_ep(const moe_config_t* c, int64_t T_global, int world) {
+    moe_status_t st = check_dp(c, T_global);
+    if (st != MOE_OK) return st;
+    if (world < 1 || c->E % world != 0) return MOE_ERR_INVALID_ARG;
+    if (world > kMaxRanks) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+Plan plan_ep(const moe_config_t* c, int64_t T_global, int world) {
+    return plan_rows(c, ep_recv_rows(c, T_global, world), false);
 }
 
 moe_status_t check_ws_plan(const Plan& pl, const void* ws, size_t ws_bytes) {
@@ -384,6 +407,7 @@ const char* moe_status_string(moe_status_t status) {
         case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or smaller than moe_workspace_size";
         case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
         case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait gave up";
+        case MOE_ERR_RANGE: return "MOE_ERR_RANGE: a device-side bounds check refused a row (inconsistent counts)";
     }
     return "MOE_ERR_UNKNOWN";
 }
@@ -571,25 +595,42 @@ moe_status_t moe_dp_max_rows(const moe_config_t* cfg, int64_t T_global, int64_t*
     return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Router and top-k of one slice of a sharded batch, with the slice's
+// per-expert counts and probability sums (the data- and expert-parallel calls).
+moe_status_t route_slice(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, const float* logits_in,
+                         moe_outputs_t* o, int32_t* local_counts, double* local_psum, void* ws, size_t ws_bytes,
+                         const Plan& pl, cudaStream_t stream) {
+    moe_status_t st = check_weights(cfg, weights, logits_in == nullptr, false);
+    if (st != MOE_OK) return st;
+    if (o == nullptr || o->offsets == nullptr || local_counts == nullptr || local_psum == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->topk_idx == nullptr || o->topk_w == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    ScanArgs sa = scan_args(cfg, local_counts, o->offsets, nullptr, nullptr, nullptr, true, ws, pl);
+    sa.cap = 0x7fffffff;        // local totals only; the capacity is applied by the second phase
+    sa.psum_total = local_psum;
+    if (cfg->T == 0) return from_cuda(launch_dispatch_scan(sa, stream));
+    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, nullptr, o->topk_idx, o->topk_w,
+                      o->logits_out, o->probs_out, ws, pl, stream, &sa);
+}
+
+}  // namespace
+
+extern "C" {
+
 moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_weights_t* weights, const void* x,
                           const float* logits_in, moe_outputs_t* o, int32_t* local_counts, double* local_psum,
                           void* ws, size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
     if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
-    if ((st = check_weights(cfg, weights, logits_in == nullptr, false)) != MOE_OK) return st;
-    if (o == nullptr || o->offsets == nullptr || local_counts == nullptr || local_psum == nullptr)
-        return MOE_ERR_INVALID_ARG;
-    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->topk_idx == nullptr || o->topk_w == nullptr))
-        return MOE_ERR_INVALID_ARG;
-    const Plan pl = plan_rows(cfg, dp_rows(cfg, T_global));
-    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
-    ScanArgs sa = scan_args(cfg, local_counts, o->offsets, nullptr, nullptr, nullptr, true, ws, pl);
-    sa.cap = 0x7fffffff;        // local totals only; the capacity is applied in moe_dp_finish
-    sa.psum_total = local_psum;
-    if (cfg->T == 0) return from_cuda(launch_dispatch_scan(sa, stream));
-    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, nullptr, o->topk_idx, o->topk_w,
-                      o->logits_out, o->probs_out, ws, pl, stream, &sa);
+    return route_slice(cfg, weights, x, logits_in, o, local_counts, local_psum, ws, ws_bytes,
+                       plan_rows(cfg, dp_rows(cfg, T_global)), stream);
 }
 
 moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
@@ -649,6 +690,204 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
                        cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
 }
 
+moe_status_t moe_ep_recv_rows(const moe_config_t* cfg, int64_t T_global, int32_t world, int64_t* rows) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    if (rows == nullptr) return MOE_ERR_INVALID_ARG;
+    *rows = ep_recv_rows(cfg, T_global, world);
+    return MOE_OK;
+}
+
+moe_status_t moe_ep_workspace_size(const moe_config_t* cfg, int64_t T_global, int32_t world, size_t* bytes) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+    *bytes = plan_ep(cfg, T_global, world).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t world, const moe_weights_t* weights,
+                          const void* x, const float* logits_in, moe_outputs_t* o, int32_t* local_counts,
+                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    return route_slice(cfg, weights, x, logits_in, o, local_counts, local_psum, ws, ws_bytes,
+                       plan_ep(cfg, T_global, world), stream);
+}
+
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
+                             const double* all_psum, int32_t world, int32_t rank, const void* x,
+                             void* const* x_recv, moe_outputs_t* o, int32_t* recv_offsets, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    if (rank < 0 || rank >= world || all_counts == nullptr || all_psum == nullptr || x_recv == nullptr ||
+        recv_offsets == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    for (int r = 0; r < world; ++r)
+        if (x_recv[r] == nullptr || !aligned16(x_recv[r])) return MOE_ERR_INVALID_ARG;
+    if (o == nullptr || o->counts == nullptr || o->offsets == nullptr || o->f == nullptr || o->p == nullptr ||
+        o->l_aux == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->topk_idx == nullptr || o->slot == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const Plan pl = plan_ep(cfg, T_global, world);
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    int32_t* dest_off = reinterpret_cast<int32_t*>(at(ws, pl.ep_dest));
+    int32_t* cap_e = reinterpret_cast<int32_t*>(at(ws, pl.cap_e));
+    EpPrepareArgs ep;
+    ep.all_counts = all_counts;
+    ep.all_psum = all_psum;
+    ep.world = world;
+    ep.rank = rank;
+    ep.E = cfg->E;
+    ep.e_per_rank = cfg->E / world;
+    ep.k = cfg->k;
+    ep.cap = (int)dp_cap_used(cfg, T_global);
+    ep.T_global = T_global;
+    ep.T_local = cfg->T;
+    ep.recv_rows = pl.rows;
+    ep.alpha = cfg->aux_alpha;
+    ep.cap_e = cap_e;
+    ep.dest_off = dest_off;
+    ep.recv_offsets = recv_offsets;
+    ep.offsets = o->offsets;
+    ep.counts = o->counts;
+    ep.f = o->f;
+    ep.p = o->p;
+    ep.l_aux = o->l_aux;
+    ep.shared_off = cfg->n_shared > 0 ? reinterpret_cast<int32_t*>(at(ws, pl.shared_off)) : nullptr;
+    ep.st = status_of(ws);
+    if (launch_ep_prepare(ep, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cfg->T == 0) return MOE_OK;
+    ScatterArgs xa;
+    xa.topk_idx = o->topk_idx;
+    xa.chunk_base = reinterpret_cast<const int32_t*>(at(ws, pl.base));
+    xa.offsets = dest_off;
+    xa.slot = o->slot;
+    xa.src_assign = nullptr;
+    xa.x = x;
+    xa.x_perm = nullptr;
+    xa.cap_e = cap_e;
+    xa.T = cfg->T;
+    xa.E = cfg->E;
+    xa.k = cfg->k;
+    xa.cap = 0;
+    xa.nchunk = pl.nchunk;
+    xa.row_bytes = (int)(cfg->d * elem_size(cfg));
+    for (int r = 0; r < world; ++r) xa.x_dst[r] = x_recv[r];
+    xa.e_per_rank = cfg->E / world;
+    xa.row_limit = pl.rows;
+    xa.st = status_of(ws);
+    return from_cuda(launch_dispatch_scatter(xa, stream));
+}
+
+moe_status_t moe_ep_expert_ffn(const moe_config_t* cfg, int64_t T_global, int32_t world,
+                               const moe_weights_t* weights, const void* x, const void* x_recv,
+                               const int32_t* recv_offsets, void* y_recv, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    moe_config_t local = *cfg;   // this rank's experts: a pool of E/world
+    local.E = cfg->E / world;
+    if ((st = check_weights(&local, weights, false, true)) != MOE_OK) return st;
+    if (x_recv == nullptr || y_recv == nullptr || recv_offsets == nullptr || !aligned16(x_recv) || !aligned16(y_recv))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->n_shared > 0 && cfg->T > 0 && (x == nullptr || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    const Plan pl = plan_ep(cfg, T_global, world);
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    if (pl.rows > 0) {
+        st = run_ffn(&local, weights, x_recv, recv_offsets, y_recv, ws, pl, stream);
+        if (st != MOE_OK) return st;
+    }
+    if (cfg->n_shared > 0 && cfg->T > 0) {
+        // the shared experts' row offsets {0, T} were written by moe_ep_dispatch
+        auto nomark = []() { return true; };
+        int n = 0;
+        if ((st = run_shared(cfg, weights, x, ws, pl, stream, nomark, nullptr, &n)) != MOE_OK) return st;
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_ep_combine(const moe_config_t* cfg, int64_t T_global, int32_t world, const void* const* y_recv,
+                            moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_config(cfg);
+    if (st != MOE_OK) return st;
+    if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
+    if (y_recv == nullptr || o == nullptr) return MOE_ERR_INVALID_ARG;
+    for (int r = 0; r < world; ++r)
+        if (y_recv[r] == nullptr || !aligned16(y_recv[r])) return MOE_ERR_INVALID_ARG;
+    const Plan pl = plan_ep(cfg, T_global, world);
+    if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    if (cfg->T == 0) return MOE_OK;
+    if (o->out == nullptr || !aligned16(o->out) || o->slot == nullptr || o->topk_w == nullptr ||
+        o->topk_idx == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    CombineArgs a;
+    a.y_perm = nullptr;
+    a.slot = o->slot;
+    a.topk_w = o->topk_w;
+    a.out = o->out;
+    a.y_shared = cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr;
+    a.n_shared = cfg->n_shared;
+    a.T = cfg->T;
+    a.d = cfg->d;
+    a.k = cfg->k;
+    for (int r = 0; r < world; ++r) a.y_src[r] = y_recv[r];
+    a.topk_idx = o->topk_idx;
+    a.e_per_rank = cfg->E / world;
+    a.row_limit = pl.rows;
+    a.st = status_of(ws);
+    return from_cuda(launch_combine(a, cfg->dtype == MOE_DT_BF16, stream));
+}
+
+moe_status_t moe_ipc_export(const void* dev_ptr, moe_ipc_buffer_t* rec) {
+    if (dev_ptr == nullptr || rec == nullptr) return MOE_ERR_INVALID_ARG;
+    using AddressRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+    static std::atomic<AddressRangeFn> cached{nullptr};
+    AddressRangeFn fn = cached.load(std::memory_order_acquire);
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || ptr == nullptr)
+            return MOE_ERR_CUDA;
+        fn = reinterpret_cast<AddressRangeFn>(ptr);
+        cached.store(fn, std::memory_order_release);
+    }
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    const CUdeviceptr p = reinterpret_cast<CUdeviceptr>(dev_ptr);
+    if (fn(&base, &size, p) != CUDA_SUCCESS || p < base || p >= base + size) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return MOE_ERR_CUDA;
+    static_assert(sizeof(h) == sizeof(rec->handle), "IPC handle size");
+    memcpy(rec->handle, &h, sizeof(h));
+    rec->offset = (uint64_t)(p - base);
+    rec->bytes = (uint64_t)(base + size - p);
+    return MOE_OK;
+}
+
+moe_status_t moe_ipc_open(const moe_ipc_buffer_t* rec, void** dev_ptr) {
+    if (rec == nullptr || dev_ptr == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, rec->handle, sizeof(h));
+    void* base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return MOE_ERR_CUDA;
+    *dev_ptr = static_cast<uint8_t*>(base) + rec->offset;
+    return MOE_OK;
+}
+
+moe_status_t moe_ipc_close(void* dev_ptr, const moe_ipc_buffer_t* rec) {
+    if (dev_ptr == nullptr || rec == nullptr) return MOE_ERR_INVALID_ARG;
+    return from_cuda(cudaIpcCloseMemHandle(static_cast<uint8_t*>(dev_ptr) - rec->offset));
+}
+
 moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* weights, const void* x_host,
                                 void* x_dev, moe_outputs_t* o, void* out_host, float* l_aux_host, void* ws,
                                 size_t ws_bytes, cudaStream_t stream) {
@@ -675,10 +914,10 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t str
     if (cudaMemcpyAsync(words, ws, sizeof(words), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
     if (site) *site = words[1];
-    if (words[0] & kErrTimeout) {
+    if (words[0] & (kErrTimeout | kErrRange)) {
         if (cudaMemsetAsync(ws, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
-        return MOE_ERR_TIMEOUT;
+        return (words[0] & kErrTimeout) ? MOE_ERR_TIMEOUT : MOE_ERR_RANGE;
     }
     return MOE_OK;
 }

@@ -175,8 +175,57 @@ def test_workspace_size_accounts_for_buffers(lib):
     assert M.moe_forward_launch_count(M.MoEConfig(T=0, d=64, ffn=64, E=2, k=1)) == 1
 
 
+def test_expert_parallel_arguments_checked_on_host(lib):
+    """The expert-parallel calls validate world, rank and pointers before any
+    CUDA call (no GPU needed)."""
+    c = M.MoEConfig(T=64, d=128, ffn=128, E=6, k=2)
+    with pytest.raises(M.MoEError) as e:
+        M.moe_ep_recv_rows(c, 128, 4)          # E % world != 0
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+    with pytest.raises(M.MoEError) as e:
+        M.moe_ep_recv_rows(M.MoEConfig(T=64, d=128, ffn=128, E=16, k=2), 128, 16)
+    assert e.value.status == M.MOE_ERR_UNSUPPORTED
+    with pytest.raises(M.MoEError) as e:
+        M.moe_ep_recv_rows(c, 32, 2)           # T_global below the slice
+    assert e.value.status == M.MOE_ERR_INVALID_ARG
+    assert M.moe_ep_recv_rows(c, 128, 2) == min(128 * 2, 3 * O.capacity(128, 2, 6, 1.25))
+    assert M.moe_ep_recv_rows(M.MoEConfig(T=64, d=128, ffn=128, E=6, k=2, capacity_factor=0.0), 128, 3) == 256
+    assert M.moe_ep_workspace_size(c, 128, 2) < M.moe_dp_workspace_size(c, 128)
+    cfg = c.c()
+    fake = ctypes.c_void_p(1 << 20)
+    arr2 = (ctypes.c_void_p * 2)(1 << 20, 1 << 21)
+    arr_null = (ctypes.c_void_p * 2)(1 << 20, None)
+    oc = M.MoEOutputsC()
+    ws = ctypes.c_size_t(1 << 30)
+    disp = lib.moe_ep_dispatch
+    disp.argtypes = [M._CFG, ctypes.c_int64, M._P, M._P, ctypes.c_int32, ctypes.c_int32, M._P,
+                     ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(M.MoEOutputsC), M._P, M._P, ctypes.c_size_t,
+                     M._P]
+    disp.restype = ctypes.c_int
+    # rank out of range, missing counts, a null peer buffer, missing outputs: all refused before any launch
+    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 2, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert disp(ctypes.byref(cfg), 128, None, fake, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 0, fake, arr_null, ctypes.byref(oc), fake, fake, ws,
+                None) == M.MOE_ERR_INVALID_ARG
+    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+        M.MOE_ERR_INVALID_ARG
+    comb = lib.moe_ep_combine
+    comb.argtypes = [M._CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
+                     ctypes.POINTER(M.MoEOutputsC), M._P, ctypes.c_size_t, M._P]
+    comb.restype = ctypes.c_int
+    assert comb(ctypes.byref(cfg), 128, 2, arr_null, ctypes.byref(oc), fake, ws, None) == M.MOE_ERR_INVALID_ARG
+    assert comb(ctypes.byref(cfg), 128, 2, arr2, ctypes.byref(oc), None, ws, None) == M.MOE_ERR_WORKSPACE
+    ipc_open = lib.moe_ipc_open
+    ipc_open.argtypes = [M._P, M._P]
+    ipc_open.restype = ctypes.c_int
+    assert ipc_open(None, None) == M.MOE_ERR_INVALID_ARG
+    assert ctypes.sizeof(M.MoEIpcBufferC) == 80
+
+
 def test_status_strings(lib):
-    for s in range(6):
+    for s in range(7):
         assert M.moe_status_string(s).startswith("MOE_")
     assert "UNKNOWN" in M.moe_status_string(99)
 
