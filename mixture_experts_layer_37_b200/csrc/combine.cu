@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
     for (int64_t t = warp_g; t < a.T; t += nwarps) {
         int s_l = -1;
         float w_l = 0.f;
-        const uint4* y_l = Y;
+        [[maybe_unused]] const uint4* y_l = Y;
         if (lane < a.k) {
             s_l = a.slot[t * a.k + lane];
             w_l = a.topk_w[t * a.k + lane];
@@ -51,12 +51,15 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
         }
         int sj[kMaxTopK];
         float wj[kMaxTopK];
-        const uint4* yj[EP ? kMaxTopK : 1];
 #pragma unroll
         for (int j = 0; j < kMaxTopK; ++j) {
             sj[j] = __shfl_sync(0xffffffffu, s_l, j);
             wj[j] = __shfl_sync(0xffffffffu, w_l, j);
-            if constexpr (EP)
+        }
+        [[maybe_unused]] const uint4* yj[EP ? kMaxTopK : 1];
+        if constexpr (EP) {
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j)
                 yj[j] = reinterpret_cast<const uint4*>(
                     __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(y_l), j));
         }
@@ -70,18 +73,23 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
             for (int j = 0; j < a.k; j += 2) {
                 const int s0 = sj[j];
                 const int s1 = (j + 1 < a.k) ? sj[j + 1] : -1;
-                const uint4* Y0 = Y;
-                const uint4* Y1 = Y;
-                if constexpr (EP) {
-                    Y0 = yj[j];
-                    Y1 = (j + 1 < a.k) ? yj[j + 1] : Y;
-                }
                 uint4 y0[U], y1[U];
+                if constexpr (EP) {
+                    const uint4* Y0 = yj[j];
+                    const uint4* Y1 = (j + 1 < a.k) ? yj[j + 1] : Y;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const bool in = v0 + 32 * u < nvec;
-                    if (in && s0 >= 0) y0[u] = Y0[(int64_t)s0 * nvec + v0 + 32 * u];
-                    if (in && s1 >= 0) y1[u] = Y1[(int64_t)s1 * nvec + v0 + 32 * u];
+                    for (int u = 0; u < U; ++u) {
+                        const bool in = v0 + 32 * u < nvec;
+                        if (in && s0 >= 0) y0[u] = Y0[(int64_t)s0 * nvec + v0 + 32 * u];
+                        if (in && s1 >= 0) y1[u] = Y1[(int64_t)s1 * nvec + v0 + 32 * u];
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const bool in = v0 + 32 * u < nvec;
+                        if (in && s0 >= 0) y0[u] = Y[(int64_t)s0 * nvec + v0 + 32 * u];
+                        if (in && s1 >= 0) y1[u] = Y[(int64_t)s1 * nvec + v0 + 32 * u];
+                    }
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
