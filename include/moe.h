@@ -297,24 +297,31 @@ moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, 
  * §3.1), and the capacity cut then drops in the batch's token order.  Results
  * equal a single moe_forward over the whole batch (row indices local).
  *   1. moe_dp_route on every rank: router and top-k of the slice; writes the
- *      slice's per-expert counts local_counts [E] (int32, device) and
- *      probability sums local_psum [E] (float64, device).
- *   2. the caller all-gathers them in rank order into all_counts [world, E]
- *      and all_psum [world, E] (device), e.g. with NCCL.
+ *      slice's per-expert counts local_counts [E] (int32, device),
+ *      probability sums local_psum [E] (float64, device) and, if local_real
+ *      is not NULL, its number of real tokens local_real [1] (int32, device).
+ *   2. the caller all-gathers them in rank order into all_counts [world, E],
+ *      all_psum [world, E] and all_real [world] (device), e.g. with NCCL.
  *   3. moe_dp_finish on every rank: capacity left for the slice, dispatch,
  *      expert FFNs, combine; outputs->counts, f, p, l_aux are the whole
  *      batch's (identical on every rank).
+ * token_mask (DEVICE [cfg->T] uint8, or NULL) marks padding as in moe_forward:
+ * a padding token selects no expert and f and p divide by the whole batch's
+ * real tokens, the sum of all_real (all_real NULL: every token is real).
+ * With a mask, local_real must be given and exchanged.  The capacity stays
+ * that of all T_global tokens.
  * Both calls use the same workspace of moe_dp_workspace_size bytes; outputs
  * src_assign and the sorted-row buffers hold up to moe_dp_max_rows rows. */
 moe_status_t moe_dp_workspace_size(const moe_config_t* cfg, int64_t T_global, size_t* bytes);
 moe_status_t moe_dp_max_rows(const moe_config_t* cfg, int64_t T_global, int64_t* rows);
 moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_weights_t* weights, const void* x,
-                          const float* logits_in, moe_outputs_t* outputs, int32_t* local_counts,
-                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream);
+                          const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs,
+                          int32_t* local_counts, double* local_psum, int32_t* local_real, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
 moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                           const double* all_psum, int32_t world, int32_t rank, const moe_weights_t* weights,
-                           const void* x, moe_outputs_t* outputs, void* ws, size_t ws_bytes,
-                           cudaStream_t stream);
+                           const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank,
+                           const moe_weights_t* weights, const void* x, moe_outputs_t* outputs, void* ws,
+                           size_t ws_bytes, cudaStream_t stream);
 
 /* ---- Expert parallelism: experts sharded over ranks --------------------
  * "Hand-building a LLaMA4-MoE" §2.5 and the MoE-basics page §4.1: each GPU
@@ -341,10 +348,12 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
  * all-to-alls are fused into the scatter and the weighted sum.
  *
  * Sequence on every rank (the same steps on all ranks, even with no rows):
- *   1. moe_ep_route: router and top-k of the slice, local_counts [E] int32
- *      and local_psum [E] float64 (device).
- *   2. all-gather local_counts / local_psum in rank order into all_counts
- *      [world, E] / all_psum [world, E] (e.g. NCCL).
+ *   1. moe_ep_route: router and top-k of the slice, local_counts [E] int32,
+ *      local_psum [E] float64 and local_real [1] int32 (device; as in
+ *      moe_dp_route, including the padding mask).
+ *   2. all-gather local_counts / local_psum / local_real in rank order into
+ *      all_counts [world, E] / all_psum [world, E] / all_real [world]
+ *      (e.g. NCCL).
  *   3. moe_ep_dispatch: capacity left, rows into the owners' x_recv,
  *      outputs->slot [T,k] = row in the owner's y_recv (or -1), recv_offsets
  *      [E/world + 1] = this rank's received rows per local expert, and the
@@ -357,18 +366,19 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
  *   7. moe_ep_combine: outputs->out [T,d] of the slice.
  * The receive buffers must not be reused by the next forward's step 3 before
  * every rank's step 7 finished (the all-gather of step 2 orders that).
- * All four calls use one workspace of moe_ep_workspace_size bytes per rank.
- * The padding mask is not supported here. */
+ * All four calls use one workspace of moe_ep_workspace_size bytes per rank. */
 moe_status_t moe_ep_recv_rows(const moe_config_t* cfg, int64_t T_global, int32_t world, int64_t* rows);
 moe_status_t moe_ep_workspace_size(const moe_config_t* cfg, int64_t T_global, int32_t world, size_t* bytes);
 moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t world, const moe_weights_t* weights,
-                          const void* x, const float* logits_in, moe_outputs_t* outputs, int32_t* local_counts,
-                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream);
-/* all_counts / all_psum: DEVICE [world, E] as gathered in step 2; counts that
- * do not match the routing make the kernels refuse rows (MOE_ERR_RANGE from
- * moe_check_device_status; memory stays in bounds). */
+                          const void* x, const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs,
+                          int32_t* local_counts, double* local_psum, int32_t* local_real, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
+/* all_counts / all_psum / all_real: DEVICE [world, E] / [world, E] / [world]
+ * as gathered in step 2 (all_real may be NULL: every token is real); counts
+ * that do not match the routing make the kernels refuse rows (MOE_ERR_RANGE
+ * from moe_check_device_status; memory stays in bounds). */
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                             const double* all_psum, int32_t world, int32_t rank, const void* x,
+                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank, const void* x,
                              void* const* x_recv, moe_outputs_t* outputs, int32_t* recv_offsets, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
 /* weights: the E/world local experts (and the shared experts); x: the

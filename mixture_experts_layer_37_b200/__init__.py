@@ -406,29 +406,31 @@ def moe_dp_max_rows(cfg: MoEConfig, T_global: int) -> int:
 
 
 def moe_dp_route(cfg: MoEConfig, T_global: int, weights: dict, x, outputs: dict, local_counts, local_psum,
-                 ws: Workspace, logits_in=None, stream=None) -> None:
+                 ws: Workspace, logits_in=None, stream=None, token_mask=None, local_real=None) -> None:
     L = lib()
     f = L.moe_dp_route
-    f.argtypes = [_CFG, ctypes.c_int64, ctypes.POINTER(MoEWeightsC), _P, _P, ctypes.POINTER(MoEOutputsC), _P, _P, _P,
-                  ctypes.c_size_t, _P]
+    f.argtypes = [_CFG, ctypes.c_int64, ctypes.POINTER(MoEWeightsC), _P, _P, _P, ctypes.POINTER(MoEOutputsC), _P, _P,
+                  _P, _P, ctypes.c_size_t, _P]
     f.restype = ctypes.c_int
     wc = _weights_c(weights)
     oc = _outputs_c(outputs)
-    _check(f(ctypes.byref(cfg.c()), int(T_global), ctypes.byref(wc), _ptr(x), _ptr(logits_in), ctypes.byref(oc),
-             _ptr(local_counts), _ptr(local_psum), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_route")
+    _check(f(ctypes.byref(cfg.c()), int(T_global), ctypes.byref(wc), _ptr(x), _ptr(logits_in), _ptr(token_mask),
+             ctypes.byref(oc), _ptr(local_counts), _ptr(local_psum), _ptr(local_real), ws.ptr, ws.nbytes,
+             _stream(stream)), "moe_dp_route")
 
 
 def moe_dp_finish(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: int, rank: int, weights: dict, x,
-                  outputs: dict, ws: Workspace, stream=None) -> None:
+                  outputs: dict, ws: Workspace, stream=None, all_real=None) -> None:
     L = lib()
     f = L.moe_dp_finish
-    f.argtypes = [_CFG, ctypes.c_int64, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P,
+    f.argtypes = [_CFG, ctypes.c_int64, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P,
                   ctypes.POINTER(MoEOutputsC), _P, ctypes.c_size_t, _P]
     f.restype = ctypes.c_int
     wc = _weights_c(weights)
     oc = _outputs_c(outputs)
-    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank),
-             ctypes.byref(wc), _ptr(x), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)), "moe_dp_finish")
+    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), _ptr(all_real), int(world),
+             int(rank), ctypes.byref(wc), _ptr(x), ctypes.byref(oc), ws.ptr, ws.nbytes, _stream(stream)),
+           "moe_dp_finish")
 
 
 # ---------------------------------------------------------------- expert parallelism
@@ -476,27 +478,27 @@ def moe_ep_workspace_size(cfg: MoEConfig, T_global: int, world: int) -> int:
 
 
 def moe_ep_route(cfg: MoEConfig, T_global: int, world: int, weights: dict, x, outputs: dict, local_counts,
-                 local_psum, ws: Workspace, logits_in=None, stream=None) -> None:
-    f = _ep_fn("moe_ep_route", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P, _P,
-                                ctypes.POINTER(MoEOutputsC), _P, _P, _P, ctypes.c_size_t, _P])
+                 local_psum, ws: Workspace, logits_in=None, stream=None, token_mask=None, local_real=None) -> None:
+    f = _ep_fn("moe_ep_route", [_CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(MoEWeightsC), _P, _P, _P,
+                                ctypes.POINTER(MoEOutputsC), _P, _P, _P, _P, ctypes.c_size_t, _P])
     wc = _weights_c(weights)
     oc = _outputs_c(outputs)
     _check(f(ctypes.byref(cfg.c()), int(T_global), int(world), ctypes.byref(wc), _ptr(x), _ptr(logits_in),
-             ctypes.byref(oc), _ptr(local_counts), _ptr(local_psum), ws.ptr, ws.nbytes, _stream(stream)),
-           "moe_ep_route")
+             _ptr(token_mask), ctypes.byref(oc), _ptr(local_counts), _ptr(local_psum), _ptr(local_real), ws.ptr,
+             ws.nbytes, _stream(stream)), "moe_ep_route")
 
 
 def moe_ep_dispatch(cfg: MoEConfig, T_global: int, all_counts, all_psum, world: int, rank: int, x, x_recv,
-                    outputs: dict, recv_offsets, ws: Workspace, stream=None) -> None:
+                    outputs: dict, recv_offsets, ws: Workspace, stream=None, all_real=None) -> None:
     """x_recv: every rank's receive buffer (tensors on this device, or device
     pointers this process can dereference), in rank order."""
-    f = _ep_fn("moe_ep_dispatch", [_CFG, ctypes.c_int64, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
+    f = _ep_fn("moe_ep_dispatch", [_CFG, ctypes.c_int64, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
                                    ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(MoEOutputsC), _P, _P,
                                    ctypes.c_size_t, _P])
     oc = _outputs_c(outputs)
-    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), int(world), int(rank), _ptr(x),
-             _ptr_array(x_recv), ctypes.byref(oc), _ptr(recv_offsets), ws.ptr, ws.nbytes, _stream(stream)),
-           "moe_ep_dispatch")
+    _check(f(ctypes.byref(cfg.c()), int(T_global), _ptr(all_counts), _ptr(all_psum), _ptr(all_real), int(world),
+             int(rank), _ptr(x), _ptr_array(x_recv), ctypes.byref(oc), _ptr(recv_offsets), ws.ptr, ws.nbytes,
+             _stream(stream)), "moe_ep_dispatch")
 
 
 def moe_ep_expert_ffn(cfg: MoEConfig, T_global: int, world: int, weights: dict, x, x_recv, recv_offsets, y_recv,

@@ -134,16 +134,27 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
     }
 }
 
+// The batch's real tokens (padding masked out): the ranks' counts summed in
+// rank order, or every token when no count is given.
+__device__ __forceinline__ int64_t real_tokens(const int32_t* all_real, int world, int64_t T_global) {
+    if (all_real == nullptr) return T_global;
+    int64_t n = 0;
+    for (int r = 0; r < world; ++r) n += all_real[r];
+    return n;
+}
+
 // One CTA: data-parallel shard preparation (see DpPrepareArgs).  The
 // assignment rank of this rank's tokens in the whole batch is the number of
 // assignments to the same expert on lower ranks plus the local rank, so this
 // rank may keep max(0, cap - base_e) more rows of expert e.  Sums over ranks
-// run in rank order.
+// run in rank order.  f and p divide by the batch's real tokens (padding
+// masked out); the capacity is that of all T_global tokens.
 __global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
     __shared__ int sKept[kMaxExperts];
     __shared__ int sCount[kMaxExperts];
     __shared__ double sP[kMaxExperts];
     const int e = threadIdx.x;
+    const int64_t t_real = real_tokens(a.all_real, a.world, a.T_global);
     if (e < a.E) {
         int base = 0, total = 0;
         double ps = 0.0;
@@ -158,7 +169,7 @@ __global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
         a.cap_e[e] = left;
         sKept[e] = mine < left ? mine : left;
         sCount[e] = total;
-        sP[e] = a.T_global > 0 ? ps / (double)a.T_global : 0.0;
+        sP[e] = t_real > 0 ? ps / (double)t_real : 0.0;
     }
     __syncthreads();
     if (e == 0) {
@@ -168,7 +179,7 @@ __global__ void __launch_bounds__(64) dp_prepare_kernel(DpPrepareArgs a) {
             a.offsets[i] = off;
             off += sKept[i];
             a.counts[i] = sCount[i];
-            const double f = a.T_global > 0 ? (double)sCount[i] / ((double)a.T_global * a.k) : 0.0;
+            const double f = t_real > 0 ? (double)sCount[i] / ((double)t_real * a.k) : 0.0;
             a.f[i] = (float)f;
             a.p[i] = (float)sP[i];
             l += f * sP[i];
@@ -198,6 +209,7 @@ __global__ void __launch_bounds__(64) ep_prepare_kernel(EpPrepareArgs a) {
     __shared__ double sP[kMaxExperts];
     __shared__ int sBad;
     const int e = threadIdx.x;
+    const int64_t t_real = real_tokens(a.all_real, a.world, a.T_global);
     if (e == 0) sBad = 0;
     __syncthreads();
     if (e < a.E) {
@@ -213,7 +225,7 @@ __global__ void __launch_bounds__(64) ep_prepare_kernel(EpPrepareArgs a) {
         sBefore[e] = base;
         sTotal[e] = total;
         sMine[e] = a.all_counts[(int64_t)a.rank * a.E + e];
-        sP[e] = a.T_global > 0 ? ps / (double)a.T_global : 0.0;
+        sP[e] = t_real > 0 ? ps / (double)t_real : 0.0;
     }
     __syncthreads();
     if (e == 0) {
@@ -246,7 +258,7 @@ __global__ void __launch_bounds__(64) ep_prepare_kernel(EpPrepareArgs a) {
             off += kept;
             const int32_t cnt = ok ? (int32_t)sTotal[i] : 0;
             a.counts[i] = cnt;
-            const double f = a.T_global > 0 ? (double)cnt / ((double)a.T_global * a.k) : 0.0;
+            const double f = t_real > 0 ? (double)cnt / ((double)t_real * a.k) : 0.0;
             a.f[i] = (float)f;
             a.p[i] = (float)sP[i];
             l += f * sP[i];

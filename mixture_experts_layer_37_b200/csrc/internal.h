@@ -24,6 +24,7 @@ struct ScanArgs {
     double* psum_total = nullptr;    // [E] out or null: sum over this batch's tokens of p[t,e] (not divided)
     const int32_t* nreal = nullptr;  // [nchunk] real (unmasked) tokens per chunk, or null: every token is real
     int32_t* shared_off = nullptr;   // [2] out or null: {0, T}, the row offsets of the shared experts' GEMMs
+    int32_t* t_real_out = nullptr;   // [1] out or null: the number of real (unmasked) tokens
     int64_t T = 0;
     int nchunk = 0, E = 0, k = 0, cap = 0;
     float alpha = 0;
@@ -90,6 +91,7 @@ cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s);
 struct DpPrepareArgs {
     const int32_t* all_counts = nullptr;  // [world, E]
     const double* all_psum = nullptr;     // [world, E]
+    const int32_t* all_real = nullptr;    // [world] real tokens per rank, or null: every token is real
     int world = 0, rank = 0, E = 0, k = 0, cap = 0;
     int64_t T_global = 0;
     float alpha = 0;
@@ -113,6 +115,7 @@ cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s);
 struct EpPrepareArgs {
     const int32_t* all_counts = nullptr;  // [world, E]
     const double* all_psum = nullptr;     // [world, E]
+    const int32_t* all_real = nullptr;    // [world] real tokens per rank, or null: every token is real
     int world = 0, rank = 0, E = 0, e_per_rank = 0, k = 0, cap = 0;
     int64_t T_global = 0, T_local = 0;
     int64_t recv_rows = 0;                // rows of every receive buffer

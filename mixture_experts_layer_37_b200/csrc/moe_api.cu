@@ -602,21 +602,23 @@ namespace {
 // Router and top-k of one slice of a sharded batch, with the slice's
 // per-expert counts and probability sums (the data- and expert-parallel calls).
 moe_status_t route_slice(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, const float* logits_in,
-                         moe_outputs_t* o, int32_t* local_counts, double* local_psum, void* ws, size_t ws_bytes,
-                         const Plan& pl, cudaStream_t stream) {
+                         const uint8_t* token_mask, moe_outputs_t* o, int32_t* local_counts, double* local_psum,
+                         int32_t* local_real, void* ws, size_t ws_bytes, const Plan& pl, cudaStream_t stream) {
     moe_status_t st = check_weights(cfg, weights, logits_in == nullptr, false);
     if (st != MOE_OK) return st;
     if (o == nullptr || o->offsets == nullptr || local_counts == nullptr || local_psum == nullptr)
         return MOE_ERR_INVALID_ARG;
+    if (token_mask != nullptr && local_real == nullptr) return MOE_ERR_INVALID_ARG;  // the count must be exchanged
     if (cfg->T > 0 && (x == nullptr || !aligned16(x) || o->topk_idx == nullptr || o->topk_w == nullptr))
         return MOE_ERR_INVALID_ARG;
     if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
     ScanArgs sa = scan_args(cfg, local_counts, o->offsets, nullptr, nullptr, nullptr, true, ws, pl);
     sa.cap = 0x7fffffff;        // local totals only; the capacity is applied by the second phase
     sa.psum_total = local_psum;
+    sa.t_real_out = local_real;
     if (cfg->T == 0) return from_cuda(launch_dispatch_scan(sa, stream));
-    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, nullptr, o->topk_idx, o->topk_w,
-                      o->logits_out, o->probs_out, ws, pl, stream, &sa);
+    return run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, token_mask, o->topk_idx,
+                      o->topk_w, o->logits_out, o->probs_out, ws, pl, stream, &sa);
 }
 
 }  // namespace
@@ -624,17 +626,18 @@ moe_status_t route_slice(const moe_config_t* cfg, const moe_weights_t* weights, 
 extern "C" {
 
 moe_status_t moe_dp_route(const moe_config_t* cfg, int64_t T_global, const moe_weights_t* weights, const void* x,
-                          const float* logits_in, moe_outputs_t* o, int32_t* local_counts, double* local_psum,
-                          void* ws, size_t ws_bytes, cudaStream_t stream) {
+                          const float* logits_in, const uint8_t* token_mask, moe_outputs_t* o, int32_t* local_counts,
+                          double* local_psum, int32_t* local_real, void* ws, size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
     if ((st = check_dp(cfg, T_global)) != MOE_OK) return st;
-    return route_slice(cfg, weights, x, logits_in, o, local_counts, local_psum, ws, ws_bytes,
+    return route_slice(cfg, weights, x, logits_in, token_mask, o, local_counts, local_psum, local_real, ws, ws_bytes,
                        plan_rows(cfg, dp_rows(cfg, T_global)), stream);
 }
 
 moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                           const double* all_psum, int32_t world, int32_t rank, const moe_weights_t* weights,
+                           const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank,
+                           const moe_weights_t* weights,
                            const void* x, moe_outputs_t* o, void* ws, size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
@@ -654,6 +657,7 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
     DpPrepareArgs dp;
     dp.all_counts = all_counts;
     dp.all_psum = all_psum;
+    dp.all_real = all_real;
     dp.world = world;
     dp.rank = rank;
     dp.E = cfg->E;
@@ -709,17 +713,18 @@ moe_status_t moe_ep_workspace_size(const moe_config_t* cfg, int64_t T_global, in
 }
 
 moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t world, const moe_weights_t* weights,
-                          const void* x, const float* logits_in, moe_outputs_t* o, int32_t* local_counts,
-                          double* local_psum, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                          const void* x, const float* logits_in, const uint8_t* token_mask, moe_outputs_t* o,
+                          int32_t* local_counts, double* local_psum, int32_t* local_real, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
     if (st != MOE_OK) return st;
     if ((st = check_ep(cfg, T_global, world)) != MOE_OK) return st;
-    return route_slice(cfg, weights, x, logits_in, o, local_counts, local_psum, ws, ws_bytes,
+    return route_slice(cfg, weights, x, logits_in, token_mask, o, local_counts, local_psum, local_real, ws, ws_bytes,
                        plan_ep(cfg, T_global, world), stream);
 }
 
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                             const double* all_psum, int32_t world, int32_t rank, const void* x,
+                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank, const void* x,
                              void* const* x_recv, moe_outputs_t* o, int32_t* recv_offsets, void* ws,
                              size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
@@ -742,6 +747,7 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const in
     EpPrepareArgs ep;
     ep.all_counts = all_counts;
     ep.all_psum = all_psum;
+    ep.all_real = all_real;
     ep.world = world;
     ep.rank = rank;
     ep.E = cfg->E;

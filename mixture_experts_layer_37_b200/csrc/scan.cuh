@@ -89,6 +89,7 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
             }
             t_real = run;
         }
+        if (lane == 0 && a.t_real_out != nullptr) a.t_real_out[0] = (int32_t)t_real;
         if (lane == 0 && a.shared_off != nullptr) {
             a.shared_off[0] = 0;
             a.shared_off[1] = (int32_t)a.T;

@@ -6,9 +6,10 @@ per-expert counts and probability sums of every slice are all-gathered (the
 exchange that data-parallel MoE training does before its load-balance loss,
 "Hand-building a LLaMA4-MoE" (dpshk.com/news/5809432) §3.1), and the second
 phase on each rank keeps only the capacity left after the lower ranks'
-assignments.  The collectives are two all-gathers of E numbers per rank (NCCL
-over NVLink on GPUs); the computation before and after runs in libmoe's
-kernels (moe_dp_route, moe_dp_finish).
+assignments.  The collectives are two all-gathers per rank (NCCL over NVLink on
+GPUs): E counts plus the slice's number of real (unmasked) tokens, and E
+probability sums; the computation before and after runs in libmoe's kernels
+(moe_dp_route, moe_dp_finish).
 """
 from __future__ import annotations
 
@@ -31,9 +32,10 @@ def gather_rank_order(t: torch.Tensor, world: int, group=None) -> torch.Tensor:
 class DataParallelMoE:
     """One rank's share of a data-parallel MoE layer forward.
 
-    `route` and `finish` default to the library's two phases; tests of the
-    orchestration on CPU ranks may substitute stand-ins with the same
-    signatures."""
+    `route(x, logits_in, token_mask)` and `finish(x, all_counts, all_psum,
+    all_real)` default to the library's two phases; tests of the orchestration
+    on CPU ranks may substitute stand-ins with the same signatures.  A route
+    stand-in fills local_counts, local_psum and local_real."""
 
     def __init__(self, cfg_local: MoEConfig, weights: dict, group=None, device="cuda",
                  route: Optional[Callable] = None, finish: Optional[Callable] = None, T_global: Optional[int] = None):
@@ -55,20 +57,28 @@ class DataParallelMoE:
             rows = max(moe_dp_max_rows(cfg_local, T_global), 1)
             self.outputs["src_assign"] = torch.empty(rows, dtype=torch.int32, device=device)
             self.ws = Workspace(cfg_local, device, nbytes=moe_dp_workspace_size(cfg_local, T_global))
-        self.local_counts = torch.zeros(cfg_local.E, dtype=torch.int32, device=device)
+        # the E counts and the number of real tokens travel in one all-gather
+        self.local_stats = torch.zeros(cfg_local.E + 1, dtype=torch.int32, device=device)
+        self.local_counts = self.local_stats[:cfg_local.E]
+        self.local_real = self.local_stats[cfg_local.E:]
         self.local_psum = torch.zeros(cfg_local.E, dtype=torch.float64, device=device)
 
-    def _lib_route(self, x, logits_in):
+    def _lib_route(self, x, logits_in, token_mask):
         moe_dp_route(self.cfg, self.T_global, self.weights, x, self.outputs, self.local_counts, self.local_psum,
-                     self.ws, logits_in)
+                     self.ws, logits_in, token_mask=token_mask, local_real=self.local_real)
 
-    def _lib_finish(self, x, all_counts, all_psum):
+    def _lib_finish(self, x, all_counts, all_psum, all_real):
         moe_dp_finish(self.cfg, self.T_global, all_counts, all_psum, self.world, self.rank, self.weights, x,
-                      self.outputs, self.ws)
+                      self.outputs, self.ws, all_real=all_real)
         return self.outputs
 
-    def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None) -> dict:
-        self._route(x_local, logits_in)
-        all_counts = gather_rank_order(self.local_counts, self.world, self.group)
+    def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None,
+                token_mask: Optional[torch.Tensor] = None) -> dict:
+        """token_mask ([T_local] uint8, 0 = padding) as in moe_forward; f and p
+        then divide by the whole batch's real tokens."""
+        self._route(x_local, logits_in, token_mask)
+        stats = gather_rank_order(self.local_stats, self.world, self.group)
+        E = self.cfg.E
+        all_counts, all_real = stats[:, :E].contiguous(), stats[:, E].contiguous()
         all_psum = gather_rank_order(self.local_psum, self.world, self.group)
-        return self._finish(x_local, all_counts, all_psum)
+        return self._finish(x_local, all_counts, all_psum, all_real)

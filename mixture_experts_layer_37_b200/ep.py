@@ -12,10 +12,10 @@ stores every kept token row straight into the receive buffer of the rank that
 holds its expert, and its combine kernel loads the expert rows straight from
 the owners' output buffers, over NVLink peer mappings of the other ranks'
 buffers (CUDA IPC, exchanged once at construction).  The collectives left are
-the all-gather of E counts and E probability sums per rank (the one
-data-parallel MoE needs as well) and two barriers: the owners' GEMMs must not
-start before every rank's rows have landed, and the combine must not read
-before every owner's GEMMs are done.  Every rank takes the same steps, even
+the all-gathers of E counts plus the slice's real-token count and of E
+probability sums per rank (the ones data-parallel MoE needs as well) and two
+barriers: the owners' GEMMs must not start before every rank's rows have
+landed, and the combine must not read before every owner's GEMMs are done.  Every rank takes the same steps, even
 when it sends or receives no rows ("Hand-building a LLaMA4-MoE" §4.3: a rank
 that skips a collective deadlocks the group).
 """
@@ -47,9 +47,11 @@ class ExpertParallelMoE:
     ``weights`` holds the router (and the shared experts, if any) and this
     rank's E/world routed experts (``local_expert_weights`` slices a full set).
     ``peers`` = (x_recv list, y_recv list), every rank's receive buffers as
-    this process sees them, replaces the IPC exchange; ``phases`` (a dict with
-    route, dispatch, ffn, combine) replaces the library's four calls.  Both
-    exist for tests of the orchestration on CPU ranks."""
+    this process sees them, replaces the IPC exchange; ``phases`` replaces the
+    library's four calls: route(x, logits_in, token_mask) (fills local_counts,
+    local_psum, local_real), dispatch(x, all_counts, all_psum, all_real),
+    ffn(x), combine() -> outputs.  Both exist for tests of the orchestration
+    on CPU ranks."""
 
     def __init__(self, cfg_local: MoEConfig, weights: dict, T_global: Optional[int] = None, group=None,
                  device="cuda", peers: Optional[tuple] = None, phases: Optional[dict] = None):
@@ -66,7 +68,10 @@ class ExpertParallelMoE:
             T_global = int(t.item())
         self.T_global = T_global
         self.E_local = cfg_local.E // self.world
-        self.local_counts = torch.zeros(cfg_local.E, dtype=torch.int32, device=device)
+        # the E counts and the number of real tokens travel in one all-gather
+        self.local_stats = torch.zeros(cfg_local.E + 1, dtype=torch.int32, device=device)
+        self.local_counts = self.local_stats[:cfg_local.E]
+        self.local_real = self.local_stats[cfg_local.E:]
         self.local_psum = torch.zeros(cfg_local.E, dtype=torch.float64, device=device)
         self._opened = []
         self._flag = None
@@ -119,13 +124,13 @@ class ExpertParallelMoE:
             dist.barrier(group=self.group)
 
     # -------------------------------------------------------------- library phases
-    def _lib_route(self, x, logits_in):
+    def _lib_route(self, x, logits_in, token_mask):
         moe_ep_route(self.cfg, self.T_global, self.world, self.weights, x, self.outputs, self.local_counts,
-                     self.local_psum, self.ws, logits_in)
+                     self.local_psum, self.ws, logits_in, token_mask=token_mask, local_real=self.local_real)
 
-    def _lib_dispatch(self, x, all_counts, all_psum):
+    def _lib_dispatch(self, x, all_counts, all_psum, all_real):
         moe_ep_dispatch(self.cfg, self.T_global, all_counts, all_psum, self.world, self.rank, x, self.x_peers,
-                        self.outputs, self.recv_offsets, self.ws)
+                        self.outputs, self.recv_offsets, self.ws, all_real=all_real)
 
     def _lib_ffn(self, x):
         moe_ep_expert_ffn(self.cfg, self.T_global, self.world, self.weights, x, self.x_recv, self.recv_offsets,
@@ -136,11 +141,15 @@ class ExpertParallelMoE:
         return self.outputs
 
     # -------------------------------------------------------------- forward
-    def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None) -> dict:
-        self._route(x_local, logits_in)
-        all_counts = gather_rank_order(self.local_counts, self.world, self.group)
+    def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None,
+                token_mask: Optional[torch.Tensor] = None) -> dict:
+        """token_mask ([T_local] uint8, 0 = padding) as in moe_forward."""
+        self._route(x_local, logits_in, token_mask)
+        stats = gather_rank_order(self.local_stats, self.world, self.group)
+        E = self.cfg.E
+        all_counts, all_real = stats[:, :E].contiguous(), stats[:, E].contiguous()
         all_psum = gather_rank_order(self.local_psum, self.world, self.group)
-        self._dispatch(x_local, all_counts, all_psum)
+        self._dispatch(x_local, all_counts, all_psum, all_real)
         self._barrier()
         self._ffn(x_local)
         self._barrier()

@@ -198,18 +198,18 @@ def test_expert_parallel_arguments_checked_on_host(lib):
     oc = M.MoEOutputsC()
     ws = ctypes.c_size_t(1 << 30)
     disp = lib.moe_ep_dispatch
-    disp.argtypes = [M._CFG, ctypes.c_int64, M._P, M._P, ctypes.c_int32, ctypes.c_int32, M._P,
+    disp.argtypes = [M._CFG, ctypes.c_int64, M._P, M._P, M._P, ctypes.c_int32, ctypes.c_int32, M._P,
                      ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(M.MoEOutputsC), M._P, M._P, ctypes.c_size_t,
                      M._P]
     disp.restype = ctypes.c_int
     # rank out of range, missing counts, a null peer buffer, missing outputs: all refused before any launch
-    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 2, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+    assert disp(ctypes.byref(cfg), 128, fake, fake, None, 2, 2, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
         M.MOE_ERR_INVALID_ARG
-    assert disp(ctypes.byref(cfg), 128, None, fake, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+    assert disp(ctypes.byref(cfg), 128, None, fake, None, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
         M.MOE_ERR_INVALID_ARG
-    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 0, fake, arr_null, ctypes.byref(oc), fake, fake, ws,
+    assert disp(ctypes.byref(cfg), 128, fake, fake, None, 2, 0, fake, arr_null, ctypes.byref(oc), fake, fake, ws,
                 None) == M.MOE_ERR_INVALID_ARG
-    assert disp(ctypes.byref(cfg), 128, fake, fake, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
+    assert disp(ctypes.byref(cfg), 128, fake, fake, None, 2, 0, fake, arr2, ctypes.byref(oc), fake, fake, ws, None) == \
         M.MOE_ERR_INVALID_ARG
     comb = lib.moe_ep_combine
     comb.argtypes = [M._CFG, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p),
@@ -217,6 +217,17 @@ def test_expert_parallel_arguments_checked_on_host(lib):
     comb.restype = ctypes.c_int
     assert comb(ctypes.byref(cfg), 128, 2, arr_null, ctypes.byref(oc), fake, ws, None) == M.MOE_ERR_INVALID_ARG
     assert comb(ctypes.byref(cfg), 128, 2, arr2, ctypes.byref(oc), None, ws, None) == M.MOE_ERR_WORKSPACE
+    # a padding mask without the real-token count to exchange is refused
+    route = lib.moe_dp_route
+    route.argtypes = [M._CFG, ctypes.c_int64, ctypes.POINTER(M.MoEWeightsC), M._P, M._P, M._P,
+                      ctypes.POINTER(M.MoEOutputsC), M._P, M._P, M._P, M._P, ctypes.c_size_t, M._P]
+    route.restype = ctypes.c_int
+    w = M.MoEWeightsC()
+    w.w_router = 1 << 20
+    oc2 = M.MoEOutputsC()
+    oc2.offsets = oc2.topk_idx = oc2.topk_w = 1 << 20
+    assert route(ctypes.byref(cfg), 128, ctypes.byref(w), fake, None, fake, ctypes.byref(oc2), fake, fake, None,
+                 fake, ws, None) == M.MOE_ERR_INVALID_ARG
     ipc_open = lib.moe_ipc_open
     ipc_open.argtypes = [M._P, M._P]
     ipc_open.restype = ctypes.c_int

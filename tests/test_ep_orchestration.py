@@ -59,13 +59,16 @@ def _worker(rank, world, port, bounds, xr, yr, q):
         E, k, El, cap = wl.E, wl.k, wl.E // world, full["cap"]
         st = {}
 
-        def route(x_, logits_in):
+        def route(x_, logits_in, token_mask):
+            assert token_mask is None
             idx = full["idx"][t0:t1]
             st["idx"] = idx
             ep.local_counts.copy_(torch.from_numpy(np.bincount(idx[idx >= 0], minlength=E).astype(np.int32)))
             ep.local_psum.copy_(torch.from_numpy(full["p"][t0:t1].sum(axis=0)))
+            ep.local_real.fill_(t1 - t0)
 
-        def dispatch(x_, all_counts, all_psum):
+        def dispatch(x_, all_counts, all_psum, all_real):
+            assert all_real.tolist() == [bounds[i + 1] - bounds[i] for i in range(world)]
             ac = all_counts.numpy().astype(np.int64)
             base, total = ac[:rank].sum(axis=0), ac.sum(axis=0)
             kept_total = np.minimum(total, cap)

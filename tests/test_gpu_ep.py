@@ -24,7 +24,7 @@ import torch
 import mixture_experts_layer_37_b200 as M
 import workloads as W
 from oracle import moe_oracle as O
-from gpu_common import host_f64, out_close, sample_tokens, to_dev, weights_dev
+from gpu_common import host_f64, mask_dev, out_close, sample_tokens, to_dev, weights_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +43,8 @@ CASES = [
     (W.Workload("ep_int8", T=300, d=256, ffn=128, E=8, k=2, act="swiglu", dtype="bf16", capacity_factor=1.25,
                 weights="int8", seed=304), [0, 150, 300]),
     (W.WORKLOADS["tiny_f32"], [0, 40, 64]),
+    (W.Workload("ep_shared_pad", T=700, d=128, ffn=192, E=8, k=2, act="swiglu", dtype="bf16", capacity_factor=0.8,
+                n_shared=1, pad_fraction=0.2, seed=305), [0, 170, 171, 520, 700]),
     (W.WORKLOADS["longctx_zipf_t32768"], [i * 4096 for i in range(9)]),
 ]
 IDS = [f"{wl.name}-{len(b) - 1}" for wl, b in CASES]
@@ -54,7 +56,7 @@ def _slice_cfg(wl, t0, t1, router="auto"):
                        n_shared=wl.n_shared, weights=wl.weights)
 
 
-def run_emulated(wl, bounds, wd, x, all_counts_fn=None, fill=None):
+def run_emulated(wl, bounds, wd, x, all_counts_fn=None, fill=None, mask=None):
     """Runs the four expert-parallel calls for every emulated rank; returns the
     ranks' state.  `fill`: a value written into the receive buffers first."""
     world = len(bounds) - 1
@@ -71,21 +73,24 @@ def run_emulated(wl, bounds, wd, x, all_counts_fn=None, fill=None):
                   out=M.allocate_outputs(c),
                   ws=M.Workspace(c, nbytes=M.moe_ep_workspace_size(c, wl.T, world)),
                   lc=torch.zeros(wl.E, dtype=torch.int32, device="cuda"),
-                  lp=torch.zeros(wl.E, dtype=torch.float64, device="cuda"))
+                  lp=torch.zeros(wl.E, dtype=torch.float64, device="cuda"),
+                  lr=torch.zeros(1, dtype=torch.int32, device="cuda"))
         if fill is not None:
             st["x_recv"].fill_(fill)
             st["y_recv"].fill_(fill)
-        M.moe_ep_route(c, wl.T, world, wd, x[t0:t1], st["out"], st["lc"], st["lp"], st["ws"])
+        M.moe_ep_route(c, wl.T, world, wd, x[t0:t1], st["out"], st["lc"], st["lp"], st["ws"],
+                       token_mask=None if mask is None else mask[t0:t1], local_real=st["lr"])
         ranks.append(st)
     all_counts = torch.stack([s["lc"] for s in ranks])
     all_psum = torch.stack([s["lp"] for s in ranks])
+    all_real = torch.cat([s["lr"] for s in ranks])
     if all_counts_fn is not None:
         all_counts = all_counts_fn(all_counts)
     xr = [s["x_recv"] for s in ranks]
     yr = [s["y_recv"] for s in ranks]
     for r, s in enumerate(ranks):
         M.moe_ep_dispatch(s["cfg"], wl.T, all_counts, all_psum, world, r, x[s["t0"]:s["t1"]], xr, s["out"],
-                          s["recv_offsets"], s["ws"])
+                          s["recv_offsets"], s["ws"], all_real=all_real)
     for r, s in enumerate(ranks):
         M.moe_ep_expert_ffn(s["cfg"], wl.T, world, M.local_expert_weights(wd, world, r), x[s["t0"]:s["t1"]],
                             s["x_recv"], s["recv_offsets"], s["y_recv"], s["ws"])
@@ -107,11 +112,12 @@ def test_ep_equals_whole_batch(wl, bounds):
     inp = W.make_inputs(wl)
     wd = _device_weights(wl, inp)
     x = to_dev(inp["x"])
-    whole = M.MoELayer(M.MoEConfig.of(wl), wd).forward(x)
+    mask = mask_dev(inp)
+    whole = M.MoELayer(M.MoEConfig.of(wl), wd).forward(x, token_mask=mask)
     torch.cuda.synchronize()
     world = len(bounds) - 1
     El = wl.E // world
-    ranks = run_emulated(wl, bounds, wd, x)
+    ranks = run_emulated(wl, bounds, wd, x, mask=mask)
     for s in ranks:
         assert M.moe_check_device_status(s["ws"])[0] == M.MOE_OK
     cat = lambda n: torch.cat([s["out"][n] for s in ranks]).cpu()  # noqa: E731
