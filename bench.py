@@ -2,6 +2,7 @@
 """Benchmark of the MoE layer forward (tokens/s) through the libmoe C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+                    [--mode replicas|ep]
 
 One step = one whole layer forward (router, top-k, dispatch, expert FFNs,
 combine, aux statistics: five kernel launches) over one batch of the workload,
@@ -18,7 +19,8 @@ reported beside it.  Under torchrun each rank runs its own independent batch
 ranks.
 
 ``--impl reference`` times the CPU oracle (numpy, float64) on the host cores
-on a bounded token sample of the same workload.
+on a bounded token sample of the same workload.  ``--mode ep`` shards the
+experts over the GPUs instead (see run_ep).
 """
 from __future__ import annotations
 
@@ -50,6 +52,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: an independent batch per GPU (default); ep: experts sharded over the GPUs")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-kernel", default="auto", choices=["auto", "warp_mma", "tcgen05"])
@@ -435,6 +439,138 @@ def run_native(a):
     print(json.dumps(line), flush=True)
 
 
+def run_ep(a):
+    """--mode ep: expert parallelism.  One batch of world x T tokens, each rank
+    holding a slice of T tokens and E/world experts (ExpertParallelMoE: rows
+    stored into and loaded from the other ranks' buffers over CUDA IPC
+    mappings, NCCL for the count all-gathers and the two barriers).  Weak
+    scaling: tokens and experts per GPU stay fixed as world grows.  Steps run
+    eagerly (the collectives are host calls); the time is the maximum over
+    ranks of the summed CUDA-event step times."""
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_layer_37_b200 as M
+    import workloads as W
+    from mixture_experts_layer_37_b200.ep import ExpertParallelMoE
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    wl = W.WORKLOADS[a.workload]
+    if wl.E % world != 0 or world > M.MOE_MAX_RANKS:
+        raise SystemExit(f"--mode ep needs E % world == 0 and world <= {M.MOE_MAX_RANKS} (E={wl.E}, world={world})")
+    T, T_global = wl.T, world * wl.T
+    wlg = wl.with_(T=T_global)
+    inp = W.make_inputs(wlg)
+    El = wl.E // world
+
+    def dev(arr):
+        if arr.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(arr)).cuda()
+
+    weights = {}
+    for n in ("w_router", "shared_gate", "shared_up", "shared_down", "shared_w1", "shared_b1", "shared_w2",
+              "shared_b2"):
+        if n in inp:
+            weights[n] = dev(inp[n])
+    for n in ("w_gate", "w_up", "w_down", "w1", "b1", "w2", "b2"):
+        if n in inp:
+            weights[n] = dev(inp[n][rank * El:(rank + 1) * El])   # this rank's experts only
+    if inp.get("router_bias") is not None:
+        weights["router_bias"] = dev(np.asarray(inp["router_bias"], dtype=np.float32))
+    x = dev(inp["x"][rank * T:(rank + 1) * T])
+    cfg = M.MoEConfig(T=T, d=wl.d, ffn=wl.ffn, E=wl.E, k=wl.k, dtype=wl.dtype, act=wl.act,
+                      capacity_factor=wl.capacity_factor, aux_alpha=wl.aux_alpha, router_kernel=a.router_kernel,
+                      gemm_kernel=a.gemm_kernel, n_shared=wl.n_shared)
+    ep = ExpertParallelMoE(cfg, weights, T_global=T_global)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    evict = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+
+    def clear_l2():
+        flush.zero_()
+        evict.sum()
+
+    def make_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record()
+        return evs
+
+    for _ in range(a.warmup):
+        clear_l2()
+        ep.forward(x)
+    torch.cuda.synchronize()
+    st = M.moe_check_device_status(ep.ws)[0]
+    assert st == M.MOE_OK, M.moe_status_string(st)
+    steps = [make_events(6) for _ in range(a.steps)]
+    props = torch.cuda.get_device_properties(local)
+    dev_id = str(props.uuid) if hasattr(props, "uuid") else str(local)
+    if not dev_id.startswith("GPU-") and len(dev_id) > 8:
+        dev_id = "GPU-" + dev_id
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev_id)
+    time.sleep(0.2)
+    for i in range(a.steps):
+        clear_l2()
+        ep.forward(x, events=steps[i])
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop()
+    st = M.moe_check_device_status(ep.ws)[0]
+    assert st == M.MOE_OK, M.moe_status_string(st)
+    ph = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(5)] for ev in steps])
+    total_ms = float(sum(ev[0].elapsed_time(ev[5]) for ev in steps))
+    recv = int(ep.recv_offsets[-1].item())
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t[0].item())
+    value = world * T * a.steps / (total_ms / 1e3)
+    # the owner's expert FFNs (two grouped GEMMs over the received rows) against the bf16 peak
+    ffn_ms = float(ph[:, 2].mean())
+    flops = ((6 if wl.act == "swiglu" else 4) * wl.d * wl.ffn * recv
+             + wl.n_shared * (6 if wl.act == "swiglu" else 4) * wl.d * wl.ffn * T)
+    pk, pk_src = peaks()
+    achieved = flops / (ffn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "expert FFN phase of rank 0 (grouped GEMMs over the received rows)",
+                "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "peak_source": f"{pk_src} (bf16 dense burst)",
+                "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None}
+    phase_names = ["route+all-gather+dispatch", "barrier", "expert FFN", "barrier", "combine"]
+    phases = {n: round(float(ph[:, j].mean()), 4) for j, n in enumerate(phase_names)}
+    launches = (6 + 2 * wl.n_shared) * a.steps
+    ep.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, generated on host)",
+        "config": {"workload": a.workload, "T_per_gpu": T, "T_global": T_global, "d": wl.d, "ffn": wl.ffn,
+                   "E": wl.E, "experts_per_gpu": El, "k": wl.k, "act": wl.act,
+                   "capacity_factor": wl.capacity_factor, "rows_received_rank0": recv,
+                   "parallelism": f"ep{world} (experts sharded, one batch over all ranks)",
+                   "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
+                   "launch": "eager (the count all-gathers and barriers are NCCL calls)"},
+        "roofline": roofline, "phases_ms_rank0": phases,
+        "e2e": None, "e2e_note": "device-resident inputs only in this mode",
+        "gpu_launches": launches, "clocks": clocks,
+        "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(a):
     import workloads as W
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -460,6 +596,8 @@ def main():
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.mode == "ep":
+        run_ep(a)
     else:
         run_native(a)
 

@@ -21,7 +21,7 @@ that skips a collective deadlocks the group).
 """
 from __future__ import annotations
 
-from typing import Callable, Optional
+from typing import Optional
 
 import torch
 import torch.distributed as dist
@@ -142,18 +142,29 @@ class ExpertParallelMoE:
 
     # -------------------------------------------------------------- forward
     def forward(self, x_local: torch.Tensor, logits_in: Optional[torch.Tensor] = None,
-                token_mask: Optional[torch.Tensor] = None) -> dict:
-        """token_mask ([T_local] uint8, 0 = padding) as in moe_forward."""
+                token_mask: Optional[torch.Tensor] = None, events: Optional[list] = None) -> dict:
+        """token_mask ([T_local] uint8, 0 = padding) as in moe_forward.
+        events: 6 CUDA events recorded on the current stream at the phase
+        boundaries (start, after the dispatch, after the first barrier, after
+        the expert FFNs, after the second barrier, after the combine)."""
+        mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        mark(0)
         self._route(x_local, logits_in, token_mask)
         stats = gather_rank_order(self.local_stats, self.world, self.group)
         E = self.cfg.E
         all_counts, all_real = stats[:, :E].contiguous(), stats[:, E].contiguous()
         all_psum = gather_rank_order(self.local_psum, self.world, self.group)
         self._dispatch(x_local, all_counts, all_psum, all_real)
+        mark(1)
         self._barrier()
+        mark(2)
         self._ffn(x_local)
+        mark(3)
         self._barrier()
-        return self._combine()
+        mark(4)
+        out = self._combine()
+        mark(5)
+        return out
 
     def close(self) -> None:
         """Unmaps the peers' buffers once no rank can still read or write them."""
