@@ -545,7 +545,7 @@ def run_ep(a):
     roofline = {"bound": "tensor", "kernel": "expert FFN phase of rank 0 (grouped GEMMs over the received rows)",
                 "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "peak_source": f"{pk_src} (bf16 dense burst)",
                 "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None}
-    phase_names = ["route+all-gather+dispatch", "barrier", "expert FFN", "barrier", "combine"]
+    phase_names = ["route+all-gather+dispatch", "barrier_before_ffn", "expert FFN", "barrier_before_combine", "combine"]
     phases = {n: round(float(ph[:, j].mean()), 4) for j, n in enumerate(phase_names)}
     launches = (6 + 2 * wl.n_shared) * a.steps
     ep.close()

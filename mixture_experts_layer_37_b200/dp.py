@@ -6,10 +6,10 @@ per-expert counts and probability sums of every slice are all-gathered (the
 exchange that data-parallel MoE training does before its load-balance loss,
 "Hand-building a LLaMA4-MoE" (dpshk.com/news/5809432) §3.1), and the second
 phase on each rank keeps only the capacity left after the lower ranks'
-assignments.  The collectives are two all-gathers per rank (NCCL over NVLink on
-GPUs): E counts plus the slice's number of real (unmasked) tokens, and E
-probability sums; the computation before and after runs in libmoe's kernels
-(moe_dp_route, moe_dp_finish).
+assignments.  The one collective is an all-gather (NCCL over NVLink on GPUs)
+of each slice's statistics, packed in one buffer: E fp64 probability sums, E
+int32 counts and the int32 number of real (unmasked) tokens.  The computation
+before and after runs in libmoe's kernels (moe_dp_route, moe_dp_finish).
 """
 from __future__ import annotations
 
@@ -23,10 +23,36 @@ from . import (MoEConfig, Workspace, allocate_outputs, moe_dp_finish, moe_dp_max
 
 
 def gather_rank_order(t: torch.Tensor, world: int, group=None) -> torch.Tensor:
-    """[world, *t.shape] with rank r's tensor in row r."""
-    parts = [torch.empty_like(t) for _ in range(world)]
-    dist.all_gather(parts, t.contiguous(), group=group)
-    return torch.stack(parts)
+    """[world, *t.shape] with rank r's tensor in row r (through host memory
+    when the backend cannot gather device tensors)."""
+    staged = t.is_cuda and dist.get_backend(group) != "nccl"
+    src = t.cpu() if staged else t.contiguous()
+    parts = [torch.empty_like(src) for _ in range(world)]
+    dist.all_gather(parts, src, group=group)
+    out = torch.stack(parts)
+    return out.to(t.device) if staged else out
+
+
+class SliceStats:
+    """One slice's routing statistics in a single device buffer, so that one
+    all-gather carries them: E fp64 probability sums, then E int32 expert
+    counts and the int32 number of real tokens.  `psum`, `counts` and `real`
+    are views into the buffer that the route call fills."""
+
+    def __init__(self, E: int, device):
+        self.E = E
+        self.buf = torch.zeros(8 * E + 4 * (E + 1), dtype=torch.uint8, device=device)
+        self.psum = self.buf[:8 * E].view(torch.float64)
+        ints = self.buf[8 * E:].view(torch.int32)
+        self.counts, self.real = ints[:E], ints[E:]
+
+    def gather(self, world: int, group=None) -> tuple:
+        """(all_counts [world, E] int32, all_psum [world, E] fp64, all_real [world] int32), rank order."""
+        allb = gather_rank_order(self.buf, world, group)
+        E = self.E
+        psum = allb[:, :8 * E].contiguous().view(torch.float64)
+        ints = allb[:, 8 * E:].contiguous().view(torch.int32)
+        return ints[:, :E].contiguous(), psum, ints[:, E].contiguous()
 
 
 class DataParallelMoE:
@@ -57,11 +83,8 @@ class DataParallelMoE:
             rows = max(moe_dp_max_rows(cfg_local, T_global), 1)
             self.outputs["src_assign"] = torch.empty(rows, dtype=torch.int32, device=device)
             self.ws = Workspace(cfg_local, device, nbytes=moe_dp_workspace_size(cfg_local, T_global))
-        # the E counts and the number of real tokens travel in one all-gather
-        self.local_stats = torch.zeros(cfg_local.E + 1, dtype=torch.int32, device=device)
-        self.local_counts = self.local_stats[:cfg_local.E]
-        self.local_real = self.local_stats[cfg_local.E:]
-        self.local_psum = torch.zeros(cfg_local.E, dtype=torch.float64, device=device)
+        self.stats = SliceStats(cfg_local.E, device)
+        self.local_counts, self.local_psum, self.local_real = self.stats.counts, self.stats.psum, self.stats.real
 
     def _lib_route(self, x, logits_in, token_mask):
         moe_dp_route(self.cfg, self.T_global, self.weights, x, self.outputs, self.local_counts, self.local_psum,
@@ -77,8 +100,5 @@ class DataParallelMoE:
         """token_mask ([T_local] uint8, 0 = padding) as in moe_forward; f and p
         then divide by the whole batch's real tokens."""
         self._route(x_local, logits_in, token_mask)
-        stats = gather_rank_order(self.local_stats, self.world, self.group)
-        E = self.cfg.E
-        all_counts, all_real = stats[:, :E].contiguous(), stats[:, E].contiguous()
-        all_psum = gather_rank_order(self.local_psum, self.world, self.group)
+        all_counts, all_psum, all_real = self.stats.gather(self.world, self.group)
         return self._finish(x_local, all_counts, all_psum, all_real)

@@ -12,9 +12,9 @@ stores every kept token row straight into the receive buffer of the rank that
 holds its expert, and its combine kernel loads the expert rows straight from
 the owners' output buffers, over NVLink peer mappings of the other ranks'
 buffers (CUDA IPC, exchanged once at construction).  The collectives left are
-the all-gathers of E counts plus the slice's real-token count and of E
-probability sums per rank (the ones data-parallel MoE needs as well) and two
-barriers: the owners' GEMMs must not start before every rank's rows have
+one all-gather of each slice's statistics (E probability sums, E counts and
+the real-token count, packed in one buffer: the one data-parallel MoE needs as
+well) and two barriers: the owners' GEMMs must not start before every rank's rows have
 landed, and the combine must not read before every owner's GEMMs are done.  Every rank takes the same steps, even
 when it sends or receives no rows ("Hand-building a LLaMA4-MoE" §4.3: a rank
 that skips a collective deadlocks the group).
@@ -28,17 +28,7 @@ import torch.distributed as dist
 
 from . import (MoEConfig, Workspace, allocate_outputs, moe_ep_combine, moe_ep_dispatch, moe_ep_expert_ffn,
                moe_ep_recv_rows, moe_ep_route, moe_ep_workspace_size, moe_ipc_close, moe_ipc_export, moe_ipc_open)
-
-
-def gather_rank_order(t: torch.Tensor, world: int, group=None) -> torch.Tensor:
-    """[world, *t.shape] with rank r's tensor in row r (through host memory
-    when the backend cannot gather device tensors)."""
-    staged = t.is_cuda and dist.get_backend(group) != "nccl"
-    src = t.cpu() if staged else t.contiguous()
-    parts = [torch.empty_like(src) for _ in range(world)]
-    dist.all_gather(parts, src, group=group)
-    out = torch.stack(parts)
-    return out.to(t.device) if staged else out
+from .dp import SliceStats
 
 
 class ExpertParallelMoE:
@@ -68,11 +58,8 @@ class ExpertParallelMoE:
             T_global = int(t.item())
         self.T_global = T_global
         self.E_local = cfg_local.E // self.world
-        # the E counts and the number of real tokens travel in one all-gather
-        self.local_stats = torch.zeros(cfg_local.E + 1, dtype=torch.int32, device=device)
-        self.local_counts = self.local_stats[:cfg_local.E]
-        self.local_real = self.local_stats[cfg_local.E:]
-        self.local_psum = torch.zeros(cfg_local.E, dtype=torch.float64, device=device)
+        self.stats = SliceStats(cfg_local.E, device)
+        self.local_counts, self.local_psum, self.local_real = self.stats.counts, self.stats.psum, self.stats.real
         self._opened = []
         self._flag = None
         ph = phases or {}
@@ -150,10 +137,7 @@ class ExpertParallelMoE:
         mark = (lambda i: events[i].record()) if events is not None else (lambda i: None)
         mark(0)
         self._route(x_local, logits_in, token_mask)
-        stats = gather_rank_order(self.local_stats, self.world, self.group)
-        E = self.cfg.E
-        all_counts, all_real = stats[:, :E].contiguous(), stats[:, E].contiguous()
-        all_psum = gather_rank_order(self.local_psum, self.world, self.group)
+        all_counts, all_psum, all_real = self.stats.gather(self.world, self.group)
         self._dispatch(x_local, all_counts, all_psum, all_real)
         mark(1)
         self._barrier()
