@@ -41,18 +41,23 @@ class SliceStats:
 
     def __init__(self, E: int, device):
         self.E = E
-        self.buf = torch.zeros(8 * E + 4 * (E + 1), dtype=torch.uint8, device=device)
+        nbytes = (8 * E + 4 * (E + 1) + 7) // 8 * 8  # rows of the gathered buffer stay 8-byte multiples
+        self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.psum = self.buf[:8 * E].view(torch.float64)
-        ints = self.buf[8 * E:].view(torch.int32)
+        ints = self.buf[8 * E:8 * E + 4 * (E + 1)].view(torch.int32)
         self.counts, self.real = ints[:E], ints[E:]
 
-    def gather(self, world: int, group=None) -> tuple:
-        """(all_counts [world, E] int32, all_psum [world, E] fp64, all_real [world] int32), rank order."""
-        allb = gather_rank_order(self.buf, world, group)
-        E = self.E
-        psum = allb[:, :8 * E].contiguous().view(torch.float64)
-        ints = allb[:, 8 * E:].contiguous().view(torch.int32)
+    @staticmethod
+    def unpack(allb: torch.Tensor, E: int) -> tuple:
+        """(all_counts [world, E] int32, all_psum [world, E] fp64, all_real [world] int32)
+        from the gathered buffers [world, nbytes]."""
+        psum = allb[:, :8 * E].clone().view(torch.float64)
+        ints = allb[:, 8 * E:8 * E + 4 * (E + 1)].clone().view(torch.int32)
         return ints[:, :E].contiguous(), psum, ints[:, E].contiguous()
+
+    def gather(self, world: int, group=None) -> tuple:
+        """The unpacked statistics of every rank, in rank order."""
+        return SliceStats.unpack(gather_rank_order(self.buf, world, group), self.E)
 
 
 class DataParallelMoE:

@@ -126,3 +126,24 @@ def test_sharded_batch_equals_whole_batch(bounds, pad):
         np.testing.assert_allclose(f, full["f"], rtol=1e-15)
         np.testing.assert_allclose(p, full["p_mean"], rtol=1e-12)
         assert abs(l - full["l_aux"]) <= 1e-12 * abs(full["l_aux"])
+
+
+@pytest.mark.parametrize("world,E", [(1, 8), (2, 6), (3, 5), (1, 64)])
+def test_slice_stats_pack_and_unpack(world, E):
+    """The packed per-slice statistics (fp64 sums, int32 counts, int32 real
+    tokens) come back exactly from gathered rows, also for a single rank."""
+    from mixture_experts_layer_37_b200.dp import SliceStats
+    rows = []
+    for r in range(world):
+        st = SliceStats(E, "cpu")
+        st.psum.copy_(torch.arange(E, dtype=torch.float64) * 0.25 + r)
+        st.counts.copy_(torch.arange(E, dtype=torch.int32) * 3 + r)
+        st.real.fill_(100 + r)
+        assert st.buf.numel() % 8 == 0
+        rows.append(st.buf.clone())
+    counts, psum, real = SliceStats.unpack(torch.stack(rows), E)
+    for r in range(world):
+        assert torch.equal(psum[r], torch.arange(E, dtype=torch.float64) * 0.25 + r)
+        assert torch.equal(counts[r], torch.arange(E, dtype=torch.int32) * 3 + r)
+        assert int(real[r]) == 100 + r
+    assert counts.is_contiguous() and psum.is_contiguous() and real.is_contiguous()
