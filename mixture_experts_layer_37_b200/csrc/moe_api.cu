@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 #include "moe.h"
 
@@ -189,6 +191,16 @@ DevStatus status_of(void* ws) {
 }
 
 uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+// A named NVTX range over the host-side launches of one stage, for profilers
+// (for example `ncu --nvtx --nvtx-include "moe_forward/"`); without an
+// attached tool each call returns at once.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -544,23 +556,39 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     }
     void* x_perm = at(ws, pl.xperm);
     void* y_perm = at(ws, pl.yperm);
+    const NvtxRange whole("moe_forward");
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, token_mask, o->topk_idx,
-                    o->topk_w, o->logits_out, o->probs_out, ws, pl, stream, &sa);
+    {
+        const NvtxRange r("moe_forward/router");
+        st = run_router(cfg, x, weights->w_router, weights->router_logit_bias, logits_in, token_mask, o->topk_idx,
+                        o->topk_w, o->logits_out, o->probs_out, ws, pl, stream, &sa);
+    }
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
     const bool gather = gathers(cfg);
-    st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
-                     stream);
+    {
+        const NvtxRange r("moe_forward/scatter");
+        st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
+                         stream);
+    }
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
-    st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr,
-                 gather ? x : nullptr, o->src_assign);
+    {
+        const NvtxRange r("moe_forward/expert_ffn");
+        st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr,
+                     gather ? x : nullptr, o->src_assign);
+    }
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
-    if ((st = run_shared(cfg, weights, x, ws, pl, stream, mark, ev, &n)) != MOE_OK) return st;
-    st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
-                     cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
+    {
+        const NvtxRange r("moe_forward/shared_experts");
+        if ((st = run_shared(cfg, weights, x, ws, pl, stream, mark, ev, &n)) != MOE_OK) return st;
+    }
+    {
+        const NvtxRange r("moe_forward/combine");
+        st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
+                         cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
+    }
     if (st != MOE_OK) return st;
     return mark() ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -742,6 +770,7 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const in
         return MOE_ERR_INVALID_ARG;
     const Plan pl = plan_ep(cfg, T_global, world);
     if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    const NvtxRange range("moe_ep_dispatch");
     int32_t* dest_off = reinterpret_cast<int32_t*>(at(ws, pl.ep_dest));
     int32_t* cap_e = reinterpret_cast<int32_t*>(at(ws, pl.cap_e));
     EpPrepareArgs ep;
@@ -807,6 +836,7 @@ moe_status_t moe_ep_expert_ffn(const moe_config_t* cfg, int64_t T_global, int32_
     if (cfg->n_shared > 0 && cfg->T > 0 && (x == nullptr || !aligned16(x))) return MOE_ERR_INVALID_ARG;
     const Plan pl = plan_ep(cfg, T_global, world);
     if ((st = check_ws_plan(pl, ws, ws_bytes)) != MOE_OK) return st;
+    const NvtxRange range("moe_ep_expert_ffn");
     if (pl.rows > 0) {
         st = run_ffn(&local, weights, x_recv, recv_offsets, y_recv, ws, pl, stream);
         if (st != MOE_OK) return st;
@@ -834,6 +864,7 @@ moe_status_t moe_ep_combine(const moe_config_t* cfg, int64_t T_global, int32_t w
     if (o->out == nullptr || !aligned16(o->out) || o->slot == nullptr || o->topk_w == nullptr ||
         o->topk_idx == nullptr)
         return MOE_ERR_INVALID_ARG;
+    const NvtxRange range("moe_ep_combine");
     CombineArgs a;
     a.y_perm = nullptr;
     a.slot = o->slot;
