@@ -32,13 +32,13 @@ def _free_port():
     return p
 
 
-def _workload(T):
+def _workload(T, E=6):
     import workloads as W
-    return W.Workload("ep", T=T, d=16, ffn=24, E=6, k=2, act="swiglu", dtype="f32", capacity_factor=0.7,
+    return W.Workload("ep", T=T, d=16, ffn=24, E=E, k=2, act="swiglu", dtype="f32", capacity_factor=0.7,
                       zipf_router_bias=True, seed=41, w_std=0.2)
 
 
-def _worker(rank, world, port, bounds, xr, yr, q):
+def _worker(rank, world, port, bounds, E, xr, yr, q):
     import sys
     import time
     sys.path.insert(0, ROOT)
@@ -51,7 +51,7 @@ def _worker(rank, world, port, bounds, xr, yr, q):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        wl = _workload(bounds[-1])
+        wl = _workload(bounds[-1], E)
         inp = W.make_inputs(wl)
         full = O.route(wl, inp)
         x = O.to_f64(inp["x"], wl.dtype)
@@ -115,14 +115,17 @@ def _worker(rank, world, port, bounds, xr, yr, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("bounds", [[0, 120, 257], [0, 50, 51, 200], [0, 0, 90]],
-                         ids=["world2", "world3-one-token", "world2-empty-slice"])
-def test_expert_parallel_forward_equals_whole_batch(bounds):
+# the first case is the pages' own multi-process check (LLaMA4-MoE page §3.1):
+# two ranks holding two of four experts each, against the single-process layer
+@pytest.mark.parametrize("bounds,E", [([0, 60, 130], 4), ([0, 120, 257], 6), ([0, 50, 51, 200], 6),
+                                      ([0, 0, 90], 6)],
+                         ids=["world2-E4", "world2", "world3-one-token", "world2-empty-slice"])
+def test_expert_parallel_forward_equals_whole_batch(bounds, E):
     import workloads as W
     from oracle import moe_oracle as O
 
     world = len(bounds) - 1
-    wl = _workload(bounds[-1])
+    wl = _workload(bounds[-1], E)
     inp = W.make_inputs(wl)
     full = O.forward(wl, inp)
     El = wl.E // world
@@ -132,7 +135,7 @@ def test_expert_parallel_forward_equals_whole_batch(bounds):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, bounds, xr, yr, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, bounds, E, xr, yr, q)) for r in range(world)]
     for p in procs:
         p.start()
     results = {}
