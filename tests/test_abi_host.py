@@ -266,3 +266,22 @@ def test_pipeline_arguments_checked_before_any_cuda_call(lib):
     assert lib.moe_pipeline_wait(None, -1) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_pipeline_check(None, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_pipeline_destroy(None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_local_expert_weights_slices_the_expert_axis():
+    """A rank's weights under expert parallelism: its contiguous block of E/world
+    routed experts (weights, biases and INT8 scales), router and shared experts
+    as they are (reading R19: rank r holds experts [r*E/world, (r+1)*E/world))."""
+    import torch
+    E, d, F = 8, 4, 6
+    full = {"w_router": torch.randn(d, E), "w_gate": torch.randn(E, d, F), "w_up": torch.randn(E, d, F),
+            "w_down": torch.randn(E, F, d), "w_gate_scale": torch.randn(E, F), "shared_gate": torch.randn(1, d, F),
+            "b1": torch.randn(E, F)}
+    for world in (1, 2, 4, 8):
+        for r in range(world):
+            loc = M.local_expert_weights(full, world, r)
+            el = E // world
+            for n in ("w_gate", "w_up", "w_down", "w_gate_scale", "b1"):
+                assert torch.equal(loc[n], full[n][r * el:(r + 1) * el]), (n, world, r)
+                assert loc[n].is_contiguous()
+            assert loc["w_router"] is full["w_router"] and loc["shared_gate"] is full["shared_gate"]
