@@ -543,7 +543,8 @@ def run_ep(a):
     pk, pk_src = peaks()
     achieved = flops / (ffn_ms / 1e3) / 1e12
     roofline = {"bound": "tensor", "kernel": "expert FFN phase of rank 0 (grouped GEMMs over the received rows)",
-                "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "peak_source": f"{pk_src} (bf16 dense burst)",
+                "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+                "peak_source": f"{pk_src} (bf16 dense burst)",
                 "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None}
     phase_names = ["route+all-gather+dispatch", "barrier_before_ffn", "expert FFN", "barrier_before_combine", "combine"]
     phases = {n: round(float(ph[:, j].mean()), 4) for j, n in enumerate(phase_names)}

@@ -378,7 +378,8 @@ moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t wor
  * that do not match the routing make the kernels refuse rows (MOE_ERR_RANGE
  * from moe_check_device_status; memory stays in bounds). */
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank, const void* x,
+                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank,
+                             const void* x,
                              void* const* x_recv, moe_outputs_t* outputs, int32_t* recv_offsets, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
 /* weights: the E/world local experts (and the shared experts); x: the

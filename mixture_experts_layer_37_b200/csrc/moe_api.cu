@@ -752,7 +752,8 @@ moe_status_t moe_ep_route(const moe_config_t* cfg, int64_t T_global, int32_t wor
 }
 
 moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const int32_t* all_counts,
-                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank, const void* x,
+                             const double* all_psum, const int32_t* all_real, int32_t world, int32_t rank,
+                             const void* x,
                              void* const* x_recv, moe_outputs_t* o, int32_t* recv_offsets, void* ws,
                              size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_config(cfg);
