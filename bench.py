@@ -18,6 +18,12 @@ reported beside it.  Under torchrun each rank runs its own independent batch
 (weak scaling, no collective on the data path); the time is the maximum over
 ranks.
 
+With no --workload, the line is the largest single-GPU workload
+(longctx_zipf_t32768: T=32768, E=32, d=ffn=4096, capacity drops) and, at one
+GPU, carries a ``per_config`` table with the same measurements (tokens/s,
+stage times, roofline of the dominant kernel, host-buffer e2e, and the CPU
+oracle on all host cores and on one core) for all five benchmark workloads.
+
 ``--impl reference`` times the CPU oracle (numpy, float64) on the host cores
 on a bounded token sample of the same workload.  ``--mode ep`` shards the
 experts over the GPUs instead (see run_ep).
@@ -39,7 +45,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer fwd tokens/s; grouped-FFN TFLOP/s & HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "llama4moe_t4096"
+DEFAULT_WORKLOAD = "longctx_zipf_t32768"
+ALL_WORKLOADS = ("tiny_f32", "llama4moe_t4096", "flat_gelu_t8192", "longctx_zipf_t32768", "decode_t64_e64")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 FLUSH_BYTES = 256 << 20
 ORACLE_SAMPLE_TOKENS = 64
@@ -50,11 +57,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None, help=f"one workload (default {DEFAULT_WORKLOAD} plus the per-config table)")
+    ap.add_argument("--per-config-steps", type=int, default=10, help="timed steps of each other workload in per_config")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--mode", default="replicas", choices=["replicas", "ep"],
                     help="replicas: an independent batch per GPU (default); ep: experts sharded over the GPUs")
-    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=10.0, help="per oracle leg, headline workload")
+    ap.add_argument("--per-config-cpu-seconds", type=float, default=4.0, help="per oracle leg, other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-kernel", default="auto", choices=["auto", "warp_mma", "tcgen05"])
     ap.add_argument("--gemm-kernel", default="auto", choices=["auto", "one_cta", "cta_pair"])
@@ -84,29 +93,68 @@ def blas_threads() -> int:
         return 1
 
 
-def oracle_step(wl, inp, tokens):
-    """One bounded sample of the workload on the CPU oracle: routing of all
-    tokens, expert FFNs and combine for `tokens`."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample_tokens(wl) -> int:
+    """Tokens of the oracle's sub-batch per step: the largest n <= 64 (at least
+    1) whose experts' weights (decoded to float64 by the oracle for every
+    expert the sub-batch reaches, at most min(E, n*k) of them) stay near 4e8
+    values, so that one step takes a few seconds at most."""
+    per_expert = (3 if wl.act == "swiglu" else 2) * wl.d * wl.ffn
+    n = 64
+    while n > 1 and min(wl.E, n * wl.k) * per_expert > 4e8:
+        n //= 2
+    return min(n, wl.T)
+
+
+def oracle_sample(wl, inp, n: int):
+    """The first n tokens of the workload as a batch of their own (same weights):
+    x, and the padding mask when there is one, cut to n rows."""
+    sub = wl.with_(T=n)
+    si = dict(inp)
+    si["x"] = inp["x"][:n]
+    if inp.get("token_mask") is not None:
+        si["token_mask"] = inp["token_mask"][:n]
+    return sub, si
+
+
+def oracle_step(sub, si):
+    """One whole forward of the oracle (routing, capacity dispatch, expert FFNs,
+    combine, statistics) on the sub-batch."""
     from oracle import moe_oracle as O
-    r = O.route(wl, inp)
-    O.forward(wl, inp, routing=r, tokens=tokens)
+    O.forward(sub, si)
 
 
-def time_oracle(wl, inp, steps=None, seconds=None, warmup=0):
-    import numpy as np
-    tokens = np.arange(min(ORACLE_SAMPLE_TOKENS, wl.T))
-    for _ in range(warmup):
-        oracle_step(wl, inp, tokens)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(wl, inp, tokens)
-        n += 1
-        el = time.perf_counter() - t0
-        if (steps is not None and n >= steps) or (seconds is not None and el >= seconds):
-            break
-    return {"value": n * len(tokens) / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} oracle steps; each routes all T={wl.T} tokens and computes the expert FFNs and "
-                      f"combine (float64, numpy/BLAS) for {len(tokens)} of them; value = output tokens / second",
+def time_oracle(wl, inp, steps=None, seconds=None, warmup=0, threads=None):
+    """The oracle as it stands, on `threads` BLAS threads (None: all of them)."""
+    from threadpoolctl import threadpool_limits
+    n = oracle_sample_tokens(wl)
+    sub, si = oracle_sample(wl, inp, n)
+    with threadpool_limits(limits=threads):
+        cores = blas_threads()
+        for _ in range(warmup):
+            oracle_step(sub, si)
+        k, t0 = 0, time.perf_counter()
+        while True:
+            oracle_step(sub, si)
+            k += 1
+            el = time.perf_counter() - t0
+            if (steps is not None and k >= steps) or (seconds is not None and el >= seconds):
+                break
+    return {"value": k * n / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu": cpu_model(), "host_cores": os.cpu_count(),
+            "sample": f"{k} oracle steps; each a whole layer forward (float64, numpy/BLAS) of a batch of the "
+                      f"workload's first {n} tokens with its weights (capacity of that batch); "
+                      f"value = output tokens / second",
             "seconds": round(el, 3)}
 
 
@@ -180,7 +228,11 @@ def recorded_traffic(kernel: str, workload: str):
     return ent.get("bytes_per_launch")
 
 
-def run_native(a):
+def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, world: int, rank: int, local: int):
+    """Every measurement of one workload: graph-replayed and eager device
+    steps, stage times and the dominant kernel's roofline, the host-buffer e2e
+    paths, and (rank 0, one GPU) the CPU oracle on all cores and on one core.
+    Returns the JSON line's fields (on every rank; only rank 0 prints)."""
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -188,15 +240,7 @@ def run_native(a):
     import mixture_experts_layer_37_b200 as M
     import workloads as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    wl = W.WORKLOADS[a.workload]
+    wl = W.WORKLOADS[name]
     if a.n_shared is not None:
         wl = wl.with_(n_shared=a.n_shared)
     if a.pad_fraction is not None:
@@ -241,27 +285,27 @@ def run_native(a):
             e.record(stream)
         return evs
 
-    for _ in range(a.warmup):
+    for _ in range(warmup):
         clear_l2()
         layer.forward(x, token_mask=tmask)
     torch.cuda.synchronize()
     layer.check()
 
     # eager steps, for comparison: every launch issued from the host
-    eager = [make_events(nl + 1) for _ in range(a.steps)]
+    eager = [make_events(nl + 1) for _ in range(steps)]
     torch.cuda.synchronize()
-    for i in range(a.steps):
+    for i in range(steps):
         clear_l2()
         M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, eager[i], token_mask=tmask)
     torch.cuda.synchronize()
     eager_ms = float(sum(ev[0].elapsed_time(ev[nl]) for ev in eager))
 
     # the timed region: K steps captured into one graph
-    steps = [make_events(nl + 1) for _ in range(a.steps)]
+    steps = [make_events(nl + 1) for _ in range(steps)]
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        for i in range(a.steps):
+        for i in range(steps):
             clear_l2()
             M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, steps[i], token_mask=tmask)
     graph.replay()  # upload and warm the graph
@@ -289,7 +333,7 @@ def run_native(a):
         t = torch.tensor([total_ms, eager_ms], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms, eager_ms = float(t[0].item()), float(t[1].item())
-    value = world * wl.T * a.steps / (total_ms / 1e3)
+    value = world * wl.T * steps / (total_ms / 1e3)
 
     # ---------------- roofline of the dominant kernel
     R = int(layer.outputs["offsets"][-1].item())
@@ -339,7 +383,7 @@ def run_native(a):
     roofline = {"bound": bound, "kernel": f"grouped expert GEMM ({dname})" if "gemm" in dname else dname,
                 "achieved": round(achieved, 2), "peak": peak, "peak_source": f"{pk_src} ({'bf16 dense burst' if bound == 'tensor' else 'HBM copy'})",
                 "unit": unit, "frac": round(achieved / peak, 4),
-                "traffic": recorded_traffic(dname, a.workload) if "gemm" in dname and wl.weights == "native" else None}
+                "traffic": recorded_traffic(dname, name) if "gemm" in dname and wl.weights == "native" else None}
     stages = {}
     for j, n in enumerate(names):
         b, w = algo[n]
@@ -365,34 +409,34 @@ def run_native(a):
     outs_host = [torch.empty_like(xs_host[0]).pin_memory() for _ in range(depth)]
     ls_host = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(depth)]
     pipe = M.Pipeline(cfg, weights, depth=depth)
-    for i in range(max(3, a.warmup)):
+    for i in range(max(3, warmup)):
         pipe.submit(xs_host[i % depth], outs_host[i % depth], ls_host[i % depth])
     pipe.wait()
     e_start, e_end = make_events(2)  # created and recorded once here; the pipeline re-records them
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    for i in range(a.steps):
+    for i in range(steps):
         pipe.submit(xs_host[i % depth], outs_host[i % depth], ls_host[i % depth],
-                    start_event=e_start if i == 0 else None, end_event=e_end if i == a.steps - 1 else None)
+                    start_event=e_start if i == 0 else None, end_event=e_end if i == steps - 1 else None)
     pipe.wait()
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
     pipe.check()
     pipe.close()
     ref_out = layer.forward(x)["out"].cpu()  # the host-buffer paths take no padding mask
-    assert torch.equal(outs_host[(a.steps - 1) % depth], ref_out), "pipelined output differs from the forward"
+    assert torch.equal(outs_host[(steps - 1) % depth], ref_out), "pipelined output differs from the forward"
 
     # (b) one synchronous-style call per step (moe_forward_hostio: copy in,
     #     forward, copy out on one stream), L2 flushed between steps
     x_host, out_host, l_host = xs_host[0], outs_host[0], ls_host[0]
     x_dev = torch.empty_like(x)
-    e2e_ev = [make_events(2) for _ in range(a.steps)]
-    for _ in range(max(1, a.warmup // 2)):
+    e2e_ev = [make_events(2) for _ in range(steps)]
+    for _ in range(max(1, warmup // 2)):
         clear_l2()
         M.moe_forward_hostio(cfg, weights, x_host, x_dev, layer.outputs, out_host, l_host, layer.ws)
     torch.cuda.synchronize()
-    for i in range(a.steps):
+    for i in range(steps):
         clear_l2()
         e2e_ev[i][0].record(stream)
         M.moe_forward_hostio(cfg, weights, x_host, x_dev, layer.outputs, out_host, l_host, layer.ws)
@@ -406,37 +450,84 @@ def run_native(a):
     layer.check()
     bx = wl.T * wl.d * bpe
     wbytes = sum(int(v.numel() * v.element_size()) for v in weights.values())
-    e2e = {"value": round(world * wl.T * a.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+    e2e = {"value": round(world * wl.T * steps / (e2e_ms / 1e3), 1), "unit": UNIT,
            "h2d_bytes_per_step": bx, "d2h_bytes_per_step": bx + 4,
            "api": f"moe_pipeline_submit (depth {depth}): copy in, forward, copy out per step, overlapped across steps",
            "l2": f"not flushed (steps overlap); expert weights {wbytes / 2**20:.0f} MiB > L2",
-           "unpipelined": {"value": round(world * wl.T * a.steps / (serial_ms / 1e3), 1), "unit": UNIT,
+           "unpipelined": {"value": round(world * wl.T * steps / (serial_ms / 1e3), 1), "unit": UNIT,
                            "api": "moe_forward_hostio, one stream, L2 flushed between steps"}}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = time_oracle(wl, inp, seconds=a.cpu_baseline_seconds)
+        cpu = time_oracle(wl, inp, seconds=cpu_seconds)
+        one = time_oracle(wl, inp, seconds=cpu_seconds, threads=1)
+        cpu["one_core"] = {"value": one["value"], "unit": UNIT, "cores": one["cores"], "sample": one["sample"],
+                           "seconds": one["seconds"]}
 
     if world > 1:
         dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
-        "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4),
-        "eager_ms_per_step": round(eager_ms / a.steps, 4), "higher_is_better": True,
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(total_ms / steps, 4),
+        "eager_ms_per_step": round(eager_ms / steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, generated on host)",
-        "config": {"workload": a.workload, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
+        "config": {"workload": name, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
                    "act": wl.act, "capacity_factor": wl.capacity_factor, "rows_dispatched": R,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
                    "launch": "timed steps replayed from one captured CUDA graph",
                    "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel, "dispatch": a.dispatch},
-        "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * a.steps,
+        "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * steps,
         "clocks": clocks, "cpu_baseline": cpu,
     }
-    print(json.dumps(line), flush=True)
+    del layer, weights, x, flush, evict, graph
+    torch.cuda.empty_cache()
+    return line
+
+
+def per_config_entry(line: dict) -> dict:
+    """The summary of one workload's line kept in the headline's per_config table."""
+    keep = ("value", "unit", "ms_per_step", "steps", "dtype", "roofline", "stages", "clocks")
+    ent = {k: line[k] for k in keep}
+    ent["rows_dispatched"] = line["config"]["rows_dispatched"]
+    ent["e2e"] = {k: line["e2e"][k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")}
+    ent["e2e_unpipelined"] = line["e2e"]["unpipelined"]["value"]
+    cpu = line.get("cpu_baseline")
+    if cpu:
+        ent["cpu_oracle_all_cores"] = {"value": round(cpu["value"], 3), "cores": cpu["cores"]}
+        ent["cpu_oracle_one_core"] = {"value": round(cpu["one_core"]["value"], 3), "cores": 1}
+    return ent
+
+
+def run_native(a):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    head = a.workload or DEFAULT_WORKLOAD
+    line = bench_workload(a, head, a.steps, a.warmup, a.cpu_baseline_seconds, world, rank, local)
+    if a.workload is None and world == 1:
+        # the other benchmark workloads, measured the same way with fewer steps
+        table = {}
+        for name in ALL_WORKLOADS:
+            if name == head:
+                table[name] = per_config_entry(line)
+                continue
+            other = bench_workload(a, name, a.per_config_steps, max(3, min(a.warmup, 5)),
+                                   a.per_config_cpu_seconds, world, rank, local)
+            table[name] = per_config_entry(other)
+        line["per_config"] = table
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def run_ep(a):
@@ -465,7 +556,8 @@ def run_ep(a):
     os.environ.setdefault("MASTER_PORT", "29531")
     dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120),
                             device_id=torch.device("cuda", local))
-    wl = W.WORKLOADS[a.workload]
+    name = a.workload or DEFAULT_WORKLOAD
+    wl = W.WORKLOADS[name]
     if wl.E % world != 0 or world > M.MOE_MAX_RANKS:
         raise SystemExit(f"--mode ep needs E % world == 0 and world <= {M.MOE_MAX_RANKS} (E={wl.E}, world={world})")
     T, T_global = wl.T, world * wl.T
@@ -558,7 +650,7 @@ def run_ep(a):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(total_ms / a.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, generated on host)",
-        "config": {"workload": a.workload, "T_per_gpu": T, "T_global": T_global, "d": wl.d, "ffn": wl.ffn,
+        "config": {"workload": name, "T_per_gpu": T, "T_global": T_global, "d": wl.d, "ffn": wl.ffn,
                    "E": wl.E, "experts_per_gpu": El, "k": wl.k, "act": wl.act,
                    "capacity_factor": wl.capacity_factor, "rows_received_rank0": recv,
                    "parallelism": f"ep{world} (experts sharded, one batch over all ranks)",
@@ -578,13 +670,14 @@ def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = W.WORKLOADS[a.workload]
+    name = a.workload or DEFAULT_WORKLOAD
+    wl = W.WORKLOADS[name]
     inp = W.make_inputs(wl)
     res = time_oracle(wl, inp, steps=a.steps, warmup=a.warmup)
     line = {"metric": METRIC, "value": round(res["value"], 3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": round(1e3 * res["seconds"] / a.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, generated on host)",
-            "config": {"workload": a.workload, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
+            "config": {"workload": name, "T": wl.T, "d": wl.d, "ffn": wl.ffn, "E": wl.E, "k": wl.k,
                        "act": wl.act, "capacity_factor": wl.capacity_factor},
             "impl": "reference",
             "cpu_baseline": {"kind": "oracle", "cores": res["cores"], "sample": res["sample"], "value": round(res["value"], 3),

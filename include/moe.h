@@ -83,7 +83,8 @@ typedef enum {
  *                        bf16, E % 8 == 0, d % 64 == 0, else
  *                        MOE_ERR_UNSUPPORTED.
  * Fed logits (logits_in) skip the GEMM and use the warp router's softmax and
- * top-k whatever the choice. */
+ * top-k under MOE_ROUTER_AUTO and MOE_ROUTER_WARP_MMA; MOE_ROUTER_TCGEN05 with
+ * fed logits returns MOE_ERR_UNSUPPORTED (that kernel has no GEMM-free path). */
 typedef enum { MOE_ROUTER_AUTO = 0, MOE_ROUTER_WARP_MMA = 1, MOE_ROUTER_TCGEN05 = 2 } moe_router_kernel_t;
 
 /* Expert GEMM kernel (bf16; the f32 path has one kernel).  Same results bit

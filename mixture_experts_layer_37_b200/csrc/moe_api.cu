@@ -262,6 +262,10 @@ ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, flo
 moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_router, const float* bias,
                         const float* logits_in, const uint8_t* mask, int32_t* idx, float* w, float* logits_out,
                         float* probs_out, void* ws, const Plan& pl, cudaStream_t s, const ScanArgs* fused = nullptr) {
+    // the tensor-core router is a GEMM kernel: with fed logits there is no GEMM
+    // for it to run, and silently running the warp router instead would hide
+    // which kernel produced the routing
+    if (logits_in != nullptr && c->router_kernel == MOE_ROUTER_TCGEN05) return MOE_ERR_UNSUPPORTED;
     RouterArgs a;
     a.x = x;
     a.w_router = w_router;

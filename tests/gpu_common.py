@@ -67,7 +67,7 @@ def out_close(gpu, ref, dtype):
     return err <= OUT_TOL[dtype] * scale + 1e-30, err, scale
 
 
-def sample_tokens(wl, routing, n_random=256, per_expert=16, seed=0) -> np.ndarray:
+def sample_tokens(wl, routing, n_random=512, per_expert=64, seed=0) -> np.ndarray:
     """Token sample for full-size configs: the first and last `per_expert`
     kept tokens of every expert, some dropped tokens, and random tokens."""
     T, k = wl.T, wl.k

@@ -163,6 +163,13 @@ def test_null_and_workspace_errors_launch_nothing(lib):
                                None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(ctypes.byref(c), None, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_aux_stats(ctypes.byref(c), None, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    # the tensor-core router has no path for fed logits: refused, not swapped for the warp router
+    tc = M.MoEConfig(T=128, d=128, ffn=128, E=8, k=2, router_kernel="tcgen05")
+    need_tc = M.moe_workspace_size(tc)
+    assert lib.moe_router_topk(ctypes.byref(tc.c()), fake, fake, None, fake, None, fake, fake, None, None, fake,
+                               need_tc, None) == M.MOE_ERR_UNSUPPORTED
+    assert lib.moe_forward(ctypes.byref(tc.c()), ctypes.byref(w), fake, fake, None, ctypes.byref(o), fake, need_tc,
+                           None) == M.MOE_ERR_UNSUPPORTED
 
 
 def test_workspace_size_accounts_for_buffers(lib):
