@@ -301,13 +301,13 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
     eager_ms = float(sum(ev[0].elapsed_time(ev[nl]) for ev in eager))
 
     # the timed region: K steps captured into one graph
-    steps = [make_events(nl + 1) for _ in range(steps)]
+    step_ev = [make_events(nl + 1) for _ in range(steps)]
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(steps):
             clear_l2()
-            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, steps[i], token_mask=tmask)
+            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, step_ev[i], token_mask=tmask)
     graph.replay()  # upload and warm the graph
     torch.cuda.synchronize()
     layer.check()
@@ -326,8 +326,8 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
     clocks = sampler.stop()
     layer.check()
 
-    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in steps])
-    step_ms = np.array([ev[0].elapsed_time(ev[nl]) for ev in steps])
+    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in step_ev])
+    step_ms = np.array([ev[0].elapsed_time(ev[nl]) for ev in step_ev])
     total_ms = float(step_ms.sum())
     if world > 1:
         t = torch.tensor([total_ms, eager_ms], dtype=torch.float64, device="cuda")
