@@ -73,19 +73,32 @@ typedef enum {
     MOE_ACT_GELU_BIAS = 1   /* W2( gelu_erf(x W1 + b1) ) + b2 */
 } moe_act_t;
 
-/* Router kernel.  Both compute the same logits up to fp32 summation order;
- * each is batch-invariant (a token's logits do not depend on T or on the other
- * tokens), and the choice never depends on T, so neither does the routing.
+/* Router kernel.  All compute the same logits up to fp32 summation order
+ * (the two warp-MMA routers exactly the same logits); each is batch-invariant
+ * (a token's logits do not depend on T or on the other tokens), and the choice
+ * never depends on T, so neither does the routing.
  *   MOE_ROUTER_AUTO      the library's choice for the shape (currently the
- *                        warp-MMA router);
- *   MOE_ROUTER_WARP_MMA  warp-level mma.sync, 32-64 tokens per CTA, every dtype;
+ *                        resident-weight warp-MMA router, or the staged one
+ *                        where its weight slices do not fit);
+ *   MOE_ROUTER_WARP_MMA  warp-level mma.sync; bf16: the router weight resident
+ *                        in shared memory across a cluster of 2-8 CTAs, tokens
+ *                        streamed by TMA (the staged kernel for shapes whose
+ *                        slices do not fit); f32: one thread per token;
  *   MOE_ROUTER_TCGEN05   TMA + tcgen05 tensor cores + TMEM, 128-token tiles:
  *                        bf16, E % 8 == 0, d % 64 == 0, else
- *                        MOE_ERR_UNSUPPORTED.
- * Fed logits (logits_in) skip the GEMM and use the warp router's softmax and
- * top-k under MOE_ROUTER_AUTO and MOE_ROUTER_WARP_MMA; MOE_ROUTER_TCGEN05 with
- * fed logits returns MOE_ERR_UNSUPPORTED (that kernel has no GEMM-free path). */
-typedef enum { MOE_ROUTER_AUTO = 0, MOE_ROUTER_WARP_MMA = 1, MOE_ROUTER_TCGEN05 = 2 } moe_router_kernel_t;
+ *                        MOE_ERR_UNSUPPORTED;
+ *   MOE_ROUTER_WARP_MMA_STAGED  warp-level mma.sync, 32-64 tokens per CTA, the
+ *                        router weight staged in shared-memory slabs by every
+ *                        CTA (bf16; f32 as MOE_ROUTER_WARP_MMA).
+ * Fed logits (logits_in) skip the GEMM and use a warp router's softmax and
+ * top-k; MOE_ROUTER_TCGEN05 with fed logits returns MOE_ERR_UNSUPPORTED (that
+ * kernel has no GEMM-free path). */
+typedef enum {
+    MOE_ROUTER_AUTO = 0,
+    MOE_ROUTER_WARP_MMA = 1,
+    MOE_ROUTER_TCGEN05 = 2,
+    MOE_ROUTER_WARP_MMA_STAGED = 3
+} moe_router_kernel_t;
 
 /* Expert GEMM kernel (bf16; the f32 path has one kernel).  Same results bit
  * for bit: every output element is one fp32 tensor-core sum over K in the
@@ -190,11 +203,15 @@ moe_status_t moe_capacity(const moe_config_t* cfg, int64_t* cap);
 moe_status_t moe_max_rows(const moe_config_t* cfg, int64_t* rows);
 
 /* Bytes of workspace the calls below need for this config (x_perm, h, y_perm,
- * per-chunk partial histograms / probability sums, status word). */
+ * per-chunk histograms, probability sums, group bases, and a 64 KB status
+ * block at its start). */
 moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
 
-/* Clear the workspace status word.  Call once after allocating a workspace
- * (and after any MOE_ERR_TIMEOUT).  Asynchronous on `stream`. */
+/* Zero the workspace's 64 KB status block: the status word, and the counters
+ * the router and dispatch kernels add into and return to zero within every
+ * launch (per-group expert counts, real-token and arrival counts).  Call once
+ * after allocating a workspace, before its first use; a status check that
+ * reports an error clears the block again itself.  Asynchronous on `stream`. */
 moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Router + softmax + top-k + renormalisation (MoE-basics §2.1, §3.1;
@@ -241,10 +258,11 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  * must not allocate after start-up) and so cannot supply a workspace.  The
  * pages have no counterpart: this is a property of the library, not of the
  * method.  Same arguments, results and errors as moe_dispatch, minus the
- * workspace.  Its scratch (per-chunk histograms and rank bases) is a fixed
- * 1 MiB array in the library's device memory on every GPU that loads it;
- * shapes with ceil(T/32)*E > 131072 (E = 64: T > 65536) return
- * MOE_ERR_UNSUPPORTED.  The first
+ * workspace.  Its scratch (per-chunk histograms, per-group counts and rank
+ * bases) is a fixed 632 KiB array in the library's device memory on every GPU
+ * that loads it; shapes with ceil(T/32)*E > 131072 (E = 64: T > 65536) return
+ * MOE_ERR_UNSUPPORTED.  Each call clears the counts it adds into with a
+ * cudaMemsetAsync on that array (no allocation).  The first
  * call on a device looks up that array's address and should come before any
  * stream capture.  All calls on a device share the array: calls that overlap
  * on the GPU race and must be serialised by the caller. */
@@ -438,12 +456,14 @@ moe_status_t moe_forward_hostio(const moe_config_t* cfg, const moe_weights_t* we
                                 void* x_dev, moe_outputs_t* outputs, void* out_host, float* l_aux_host,
                                 void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Synchronises `stream`, then reads and clears the workspace status word.
+/* Synchronises `stream`, then reads the workspace status word.
  * Returns MOE_ERR_TIMEOUT if a bounded device wait gave up since the last
  * check (`*site`, if not NULL, receives the code of the first wait that gave
  * up), else MOE_ERR_RANGE if a device-side bounds check refused a row (the
  * expert-parallel calls given counts that do not match the routing),
- * MOE_ERR_CUDA if the synchronisation failed, else MOE_OK. */
+ * MOE_ERR_CUDA if the synchronisation failed, else MOE_OK.  After an error it
+ * zeroes the whole status block (a launch that gave up may have left its
+ * counters partly added), so the workspace is ready for the next call. */
 moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t stream, uint32_t* site);
 
 /* ---- Pipelined forwards on host-resident batches ------------------------

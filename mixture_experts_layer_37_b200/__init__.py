@@ -26,8 +26,9 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_MAX_RANKS = 8  # ranks of one expert-parallel group
 MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_ACT_SWIGLU, MOE_ACT_GELU_BIAS = 0, 1
-MOE_ROUTER_AUTO, MOE_ROUTER_WARP_MMA, MOE_ROUTER_TCGEN05 = 0, 1, 2
-ROUTER_KERNELS = {"auto": MOE_ROUTER_AUTO, "warp_mma": MOE_ROUTER_WARP_MMA, "tcgen05": MOE_ROUTER_TCGEN05}
+MOE_ROUTER_AUTO, MOE_ROUTER_WARP_MMA, MOE_ROUTER_TCGEN05, MOE_ROUTER_WARP_MMA_STAGED = 0, 1, 2, 3
+ROUTER_KERNELS = {"auto": MOE_ROUTER_AUTO, "warp_mma": MOE_ROUTER_WARP_MMA, "tcgen05": MOE_ROUTER_TCGEN05,
+                  "warp_mma_staged": MOE_ROUTER_WARP_MMA_STAGED}
 MOE_GEMM_AUTO, MOE_GEMM_ONE_CTA, MOE_GEMM_CTA_PAIR = 0, 1, 2
 GEMM_KERNELS = {"auto": MOE_GEMM_AUTO, "one_cta": MOE_GEMM_ONE_CTA, "cta_pair": MOE_GEMM_CTA_PAIR}
 MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER = 0, 1, 2
@@ -129,7 +130,7 @@ class MoEConfig:
     act: str = "swiglu"        # "swiglu" | "gelu_bias"
     capacity_factor: float = 1.25
     aux_alpha: float = 0.01
-    router_kernel: str = "auto"  # "auto" | "warp_mma" | "tcgen05"
+    router_kernel: str = "auto"  # "auto" | "warp_mma" | "tcgen05" | "warp_mma_staged"
     gemm_kernel: str = "auto"    # "auto" | "one_cta" | "cta_pair"
     dispatch: str = "auto"       # "auto" | "copy" | "gather"
     n_shared: int = 0            # shared experts, applied to every token with weight 1

@@ -17,9 +17,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["moe_api.cu", "router.cu", "router_sm100.cu", "dispatch.cu", "gemm_sm100.cu", "gemm_sm100_pair.cu", "ffn_simt.cu", "combine.cu",
+SOURCES = ["moe_api.cu", "router.cu", "router_v2.cu", "router_sm100.cu", "dispatch.cu", "gemm_sm100.cu", "gemm_sm100_pair.cu", "ffn_simt.cu", "combine.cu",
            "dispatch_noalloc.cu", "pipeline.cu", "ffn_int8.cu"]
-HEADERS = ["common.cuh", "internal.h", "scan.cuh", "gemm_common.cuh"]
+HEADERS = ["common.cuh", "internal.h", "scan.cuh", "gemm_common.cuh", "warp_mma.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-Wno-deprecated-gpu-targets"]

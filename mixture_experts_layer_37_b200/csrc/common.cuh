@@ -15,11 +15,19 @@ constexpr int kChunkTokens = 32;
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
 
-// Workspace status block: word 0 = error bits, word 1 = site of the first
-// wait that gave up, word 2 = a flag nothing ever sets (bounded-wait self-test),
-// word 4 = arrival counter of the router CTAs (the last one runs the scan; it
-// resets the counter to 0, and moe_workspace_init zeroes it).
+// Workspace status block (kStatusBlockBytes, zeroed by moe_workspace_init):
+// word 0 = error bits, word 1 = site of the first wait that gave up, word 2 =
+// a flag nothing ever sets (bounded-wait self-test), word 4 = arrival counter
+// of the router CTAs (the last one runs the scan and resets it to 0), word 5 =
+// real (unmasked) tokens counted by the router (read and reset by the scan);
+// from byte kGroupHistOffset: the per-group expert counts [E, ngroups], added
+// atomically by the router (or histogram) CTAs and returned to zero by the
+// scan that reads them.  Every launch leaves these counters at zero again.
 constexpr int kStatusCounterWord = 4;
+constexpr int kStatusRealWord = 5;
+constexpr int kStatusBlockBytes = 64 * 1024;
+constexpr int kGroupHistOffset = 4096;
+constexpr int kMaxGroupEntries = (kStatusBlockBytes - kGroupHistOffset) / 4;  // E * ngroups
 constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrRange = 2u;  // a row index failed a bounds check; the access was skipped
 // Ranks of one expert-parallel group (the GPUs of one NVSwitch node).
@@ -34,6 +42,11 @@ enum WaitSite : uint32_t {
     SITE_GEMM_PRODUCER_DRAIN = 0x106,
     SITE_SELFTEST_MBAR = 0x201,
     SITE_SELFTEST_FLAG = 0x202,
+    SITE_ROUTER_RING_EMPTY = 0x401,
+    SITE_ROUTER_RING_FULL = 0x402,
+    SITE_ROUTER_XCHG_EMPTY = 0x403,
+    SITE_ROUTER_XCHG_FULL = 0x404,
+    SITE_ROUTER_DRAIN = 0x405,
     SITE_EP_SCATTER_ROW = 0x301,
     SITE_EP_PREPARE_ROWS = 0x302,
     SITE_EP_COMBINE_ROW = 0x303,

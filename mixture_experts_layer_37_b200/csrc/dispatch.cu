@@ -9,9 +9,10 @@
 // per-expert counts, split).
 //
 // Deterministic by construction: the rank of assignment (t, j) among the
-// assignments to its expert is the chunk's base (an exclusive scan over
-// chunks of per-chunk histograms) plus the rank inside the chunk, taken from
-// warp match masks and a scan over warps; no atomic decides an order.
+// assignments to its expert is the chunk's base (the exclusive scan over
+// groups of chunks, plus the counts of the earlier chunks of its group) plus
+// the rank inside the chunk, taken from warp match masks and a scan over
+// warps; no atomic decides an order (the group counts are integer sums).
 #include "scan.cuh"
 
 namespace moe {
@@ -22,7 +23,8 @@ constexpr int kScatterWarps = kScatterThreads / 32;
 static_assert(kChunkTokens * kMaxTopK <= kScatterThreads, "one scatter CTA covers a chunk's assignments");
 
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ hist,
-                                                   int64_t T, int E, int k, int nchunk) {
+                                                   int32_t* __restrict__ group_hist, int64_t T, int E, int k,
+                                                   int nchunk, int group_chunks, int ngroups) {
     __shared__ int sHist[kMaxExperts];
     const int tid = threadIdx.x;
     if (tid < E) sHist[tid] = 0;
@@ -34,7 +36,11 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
         if (e >= 0 && e < E) atomicAdd(&sHist[e], 1);
     }
     __syncthreads();
-    if (tid < E) hist[(int64_t)tid * nchunk + blockIdx.x] = sHist[tid];
+    if (tid < E) {
+        const int n = sHist[tid];
+        hist[(int64_t)tid * nchunk + blockIdx.x] = n;
+        if (n) atomicAdd(group_hist + (int64_t)tid * ngroups + blockIdx.x / group_chunks, n);
+    }
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
@@ -70,7 +76,7 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
     if (e >= 0 && lrank == 0) sWarpBase[warp][e] = __popc(peers);
     __syncthreads();
     if (tid < E) {
-        int run = a.chunk_base[(int64_t)tid * a.nchunk + chunk];
+        int run = chunk_base_of(a.hist, a.group_base, tid, chunk, a.nchunk, a.group_chunks, a.ngroups);
         for (int w = 0; w < kScatterWarps; ++w) {
             const int c = sWarpBase[w][tid];
             sWarpBase[w][tid] = run;
@@ -284,10 +290,11 @@ cudaError_t launch_dp_prepare(const DpPrepareArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s) {
+cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int32_t* group_hist, int64_t T, int E, int k,
+                                 int group_chunks, int ngroups, cudaStream_t s) {
     const int nchunk = (int)((T + kChunkTokens - 1) / kChunkTokens);
     if (nchunk == 0) return cudaSuccess;
-    hist_kernel<<<nchunk, 256, 0, s>>>(topk_idx, hist, T, E, k, nchunk);
+    hist_kernel<<<nchunk, 256, 0, s>>>(topk_idx, hist, group_hist, T, E, k, nchunk, group_chunks, ngroups);
     return cudaGetLastError();
 }
 

@@ -9,7 +9,7 @@
 // Such a caller cannot provide the workspace that moe_dispatch needs for its
 // per-chunk histograms and rank bases.  This entry point keeps that scratch
 // in a fixed-size array in the library's own device memory instead
-// (`g_dispatch_scratch`, 1 MiB on every GPU that loads the library, held
+// (`g_dispatch_scratch`, 632 KiB on every GPU that loads the library, held
 // until the process exits).
 //
 // Limits and rules:
@@ -19,9 +19,11 @@
 //     (cudaGetSymbolAddress) with that device current; make that first call
 //     before any stream capture.
 //   - Every call on a device shares the one array, which keeps what the last
-//     call wrote.  Nothing in it has to start at zero (each call writes every
-//     entry it later reads), but calls that overlap on the GPU -- two streams,
-//     or two host threads -- race on it and give wrong results.  Serialise them.
+//     call wrote.  Nothing in it has to start at zero: each call clears the
+//     per-group counts it adds into (a cudaMemsetAsync on the array, no
+//     allocation) and writes every other entry it later reads.  Calls that
+//     overlap on the GPU -- two streams, or two host threads -- race on it and
+//     give wrong results.  Serialise them.
 //   - No cudaMalloc, cudaFree or allocating library routine is called.
 #include <mutex>
 
@@ -33,8 +35,10 @@ namespace {
 constexpr int64_t kNoAllocMaxEntries = 131072;  // ceil(T/32) * E
 constexpr int kMaxDevices = 64;
 
-// [0, kNoAllocMaxEntries): per-chunk expert histogram; [kNoAllocMaxEntries, 2x): per-chunk rank bases.
-static __device__ __align__(256) int32_t g_dispatch_scratch[2 * kNoAllocMaxEntries];
+// [0, kNoAllocMaxEntries): per-chunk expert histogram; then per-group expert
+// counts and per-group rank bases, moe::kMaxGroupEntries each.
+constexpr int64_t kScratchEntries = kNoAllocMaxEntries + 2 * (int64_t)moe::kMaxGroupEntries;
+static __device__ __align__(256) int32_t g_dispatch_scratch[kScratchEntries];
 
 std::mutex g_setup_mutex;
 int32_t* g_scratch_on_device[kMaxDevices] = {nullptr};
@@ -78,13 +82,20 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     int32_t* scratch = nullptr;
     if ((st = scratch_address(&scratch)) != MOE_OK) return st;
     int32_t* hist = scratch;
-    int32_t* chunk_base = scratch + kNoAllocMaxEntries;
+    int32_t* group_hist = scratch + kNoAllocMaxEntries;
+    int32_t* group_base = group_hist + moe::kMaxGroupEntries;
+    const int group_chunks = moe::group_chunks_for(cfg->E, nchunk);
+    const int ngroups = moe::ngroups_for(cfg->E, nchunk);
 
-    if (moe::launch_dispatch_hist(topk_idx, hist, cfg->T, cfg->E, cfg->k, stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(group_hist, 0, (size_t)ngroups * cfg->E * sizeof(int32_t), stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (moe::launch_dispatch_hist(topk_idx, hist, group_hist, cfg->T, cfg->E, cfg->k, group_chunks, ngroups, stream) !=
+        cudaSuccess)
+        return MOE_ERR_CUDA;
     moe::ScanArgs sa;
-    sa.hist = hist;
+    sa.group_hist = group_hist;
     sa.psum = nullptr;
-    sa.chunk_base = chunk_base;
+    sa.group_base = group_base;
     sa.counts = counts;
     sa.offsets = offsets;
     sa.f = nullptr;
@@ -92,7 +103,8 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     sa.l_aux = nullptr;
     sa.psum_total = nullptr;
     sa.T = cfg->T;
-    sa.nchunk = (int)nchunk;
+    sa.ngroups = ngroups;
+    sa.npsum = 0;
     sa.E = cfg->E;
     sa.k = cfg->k;
     sa.cap = (int)cap;
@@ -100,7 +112,10 @@ extern "C" moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const void
     if (moe::launch_dispatch_scan(sa, stream) != cudaSuccess) return MOE_ERR_CUDA;
     moe::ScatterArgs xa;
     xa.topk_idx = topk_idx;
-    xa.chunk_base = chunk_base;
+    xa.hist = hist;
+    xa.group_base = group_base;
+    xa.group_chunks = group_chunks;
+    xa.ngroups = ngroups;
     xa.offsets = offsets;
     xa.slot = slot;
     xa.src_assign = src_assign;

@@ -12,21 +12,35 @@
 
 namespace moe {
 
+// Chunks of kChunkTokens tokens are grouped kGroupChunks at a time for the
+// dispatch scan: the smallest power-of-two multiple of 32 chunks that keeps
+// E * ngroups within the status block's group counts.
+inline int group_chunks_for(int E, int64_t nchunk) {
+    int g = 32;
+    while ((int64_t)E * ((nchunk + g - 1) / g) > kMaxGroupEntries) g *= 2;
+    return g;
+}
+inline int ngroups_for(int E, int64_t nchunk) {
+    const int g = group_chunks_for(E, nchunk);
+    return (int)((nchunk + g - 1) / g);
+}
+
 struct ScanArgs {
-    const int32_t* hist = nullptr;   // [E, nchunk] per-chunk expert histogram
-    const double* psum = nullptr;    // [E, nchunk] per-chunk probability sums, or null (no aux stats)
-    int32_t* chunk_base = nullptr;   // [E, nchunk] out: assignments to e in earlier chunks
+    int32_t* group_hist = nullptr;   // [E, ngroups] per-group expert counts (status block); read, then reset to 0
+    const double* psum = nullptr;    // [E, npsum] partial sums of the probabilities, or null (no aux stats)
+    int32_t* group_base = nullptr;   // [E, ngroups] out: assignments to e in earlier groups
     int32_t* counts = nullptr;       // [E] out
     int32_t* offsets = nullptr;      // [E+1] out
     float* f = nullptr;              // [E] out or null
     float* p = nullptr;              // [E] out or null
     float* l_aux = nullptr;          // [1] out or null
     double* psum_total = nullptr;    // [E] out or null: sum over this batch's tokens of p[t,e] (not divided)
-    const int32_t* nreal = nullptr;  // [nchunk] real (unmasked) tokens per chunk, or null: every token is real
+    int32_t* real_counter = nullptr; // [1] real (unmasked) tokens counted by the router (read, then reset to 0),
+                                     // or null: every token is real
     int32_t* shared_off = nullptr;   // [2] out or null: {0, T}, the row offsets of the shared experts' GEMMs
     int32_t* t_real_out = nullptr;   // [1] out or null: the number of real (unmasked) tokens
     int64_t T = 0;
-    int nchunk = 0, E = 0, k = 0, cap = 0;
+    int ngroups = 0, npsum = 0, E = 0, k = 0, cap = 0;
     float alpha = 0;
 };
 
@@ -39,32 +53,43 @@ struct RouterArgs {
     float* topk_w = nullptr;           // [T, k]
     float* logits_out = nullptr;       // [T, E] or null
     float* probs_out = nullptr;        // [T, E] or null
-    int32_t* hist = nullptr;           // [E, nchunk] per-chunk expert histogram
-    double* psum = nullptr;            // [E, nchunk] per-chunk sum of probabilities
+    int32_t* hist = nullptr;           // [E, nchunk] out: per-chunk expert histogram
+    int32_t* group_hist = nullptr;     // [E, ngroups] per-group counts, added atomically (zero on entry)
+    double* psum = nullptr;            // [E, npsum] out: partial probability sums (per chunk, or per CTA)
     const uint8_t* mask = nullptr;     // [T] 0 = padding token (selects nothing, not in the sums), or null
-    int32_t* nreal = nullptr;          // [nchunk] out: real tokens per chunk (written when mask != null)
+    int32_t* real_counter = nullptr;   // [1] real tokens, added atomically (when mask != null)
     int64_t T = 0;
     int d = 0, E = 0, k = 0, nchunk = 0;
+    int group_chunks = 32, ngroups = 0;
+    int psum_cap = 0;            // columns of psum available (>= nchunk)
     int tpc = 0;                 // tokens per CTA (set by the launcher; multiple of the chunk)
     // when fuse_scan != 0: the last CTA to finish (counted on `counter`) runs
     // the dispatch scan and the aux statistics described by `scan`
     int fuse_scan = 0;
     unsigned int* counter = nullptr;
     ScanArgs scan;
-    DevStatus st;            // status word and wait limit (tensor-core router)
+    DevStatus st;            // status word and wait limit
     int kernel = 0;              // moe_router_kernel_t
 };
 cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s);
 // Tensor-core router (TMA + tcgen05 + TMEM): bf16, E % 8 == 0, no logits feed.
 bool router_tc_supported(const RouterArgs& a);
 cudaError_t launch_router_tc(const RouterArgs& a, DevStatus st, cudaStream_t s);
+// Warp-MMA router with the router weight resident across a CTA cluster (bf16):
+// same logits as the slab-staged warp-MMA router; shapes whose weight slices
+// do not fit in shared memory are not supported (the staged router takes them).
+bool router_v2_supported(const RouterArgs& a);
+cudaError_t launch_router_v2(const RouterArgs& a, cudaStream_t s);
+int router_v2_psum_columns();  // probability-sum columns the v2 router may write per expert
 
-cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int64_t T, int E, int k, cudaStream_t s);
+cudaError_t launch_dispatch_hist(const int32_t* topk_idx, int32_t* hist, int32_t* group_hist, int64_t T, int E, int k,
+                                 int group_chunks, int ngroups, cudaStream_t s);
 cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s);
 
 struct ScatterArgs {
     const int32_t* topk_idx = nullptr;    // [T, k]
-    const int32_t* chunk_base = nullptr;  // [E, nchunk]
+    const int32_t* hist = nullptr;        // [E, nchunk] per-chunk expert histogram
+    const int32_t* group_base = nullptr;  // [E, ngroups] assignments to e in earlier groups of group_chunks chunks
     const int32_t* offsets = nullptr;     // [E+1]
     int32_t* slot = nullptr;              // [T, k]
     int32_t* src_assign = nullptr;        // [R_max]
@@ -72,7 +97,7 @@ struct ScatterArgs {
     void* x_perm = nullptr;               // [R_max, d], or null: no row copies (slot / src_assign only)
     const int32_t* cap_e = nullptr;       // [E] per-expert capacity left for this batch, or null (use cap)
     int64_t T = 0;
-    int E = 0, k = 0, cap = 0, nchunk = 0;
+    int E = 0, k = 0, cap = 0, nchunk = 0, group_chunks = 32, ngroups = 0;
     int row_bytes = 0;              // d * element size (multiple of 16)
     // expert parallelism (e_per_rank > 0): the rows of expert e go to
     // x_dst[e / e_per_rank] (the receive buffer of the rank holding e, possibly

@@ -32,7 +32,7 @@ using namespace moe;
 
 uint32_t g_timeout_ms = 2000;
 
-constexpr size_t kStatusBytes = 1024;
+constexpr size_t kStatusBytes = kStatusBlockBytes;
 constexpr int kMaxShared = 8;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -46,7 +46,7 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->dtype != MOE_DT_F32 && c->dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
     if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_GELU_BIAS) return MOE_ERR_INVALID_ARG;
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
-        c->router_kernel > MOE_ROUTER_TCGEN05 || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
+        c->router_kernel > MOE_ROUTER_WARP_MMA_STAGED || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
         c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER || c->n_shared < 0 ||
         c->weight_format < MOE_WEIGHTS_NATIVE || c->weight_format > MOE_WEIGHTS_INT8)
         return MOE_ERR_INVALID_ARG;
@@ -86,9 +86,9 @@ int64_t max_rows(const moe_config_t* c) {
 }
 
 struct Plan {
-    int nchunk;
+    int nchunk, group_chunks, ngroups, psum_cols;
     int64_t rows;
-    size_t hist, psum, base, cap_e, nreal, shared_off, ep_dest, xperm, h, yperm, hs, ys, total;
+    size_t hist, psum, gbase, cap_e, shared_off, ep_dest, xperm, h, yperm, hs, ys, total;
 };
 
 // perm_buffers = false: no x_perm / y_perm (the expert-parallel calls use the
@@ -96,6 +96,10 @@ struct Plan {
 Plan plan_rows(const moe_config_t* c, int64_t rows, bool perm_buffers = true) {
     Plan p;
     p.nchunk = (int)((c->T + kChunkTokens - 1) / kChunkTokens);
+    p.group_chunks = group_chunks_for(c->E, p.nchunk);
+    p.ngroups = ngroups_for(c->E, p.nchunk);
+    // probability sums per chunk, or per CTA of the resident-weight router
+    p.psum_cols = p.nchunk > router_v2_psum_columns() ? p.nchunk : router_v2_psum_columns();
     p.rows = rows;
     const size_t s = elem_size(c);
     const size_t E = (size_t)c->E;
@@ -103,13 +107,11 @@ Plan plan_rows(const moe_config_t* c, int64_t rows, bool perm_buffers = true) {
     p.hist = off;
     off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
     p.psum = off;
-    off = align_up(off + (size_t)p.nchunk * E * 8, 1024);
-    p.base = off;
-    off = align_up(off + (size_t)p.nchunk * E * 4, 1024);
+    off = align_up(off + (size_t)p.psum_cols * E * 8, 1024);
+    p.gbase = off;
+    off = align_up(off + (size_t)p.ngroups * E * 4, 1024);
     p.cap_e = off;
     off = align_up(off + E * 4, 1024);
-    p.nreal = off;
-    off = align_up(off + (size_t)p.nchunk * 4, 1024);
     p.shared_off = off;
     off = align_up(off + 2 * 4, 1024);
     p.ep_dest = off;
@@ -238,19 +240,20 @@ moe_status_t check_weights(const moe_config_t* c, const moe_weights_t* w, bool n
 ScanArgs scan_args(const moe_config_t* c, int32_t* counts, int32_t* offsets, float* f, float* p, float* l_aux,
                    bool with_stats, void* ws, const Plan& pl) {
     ScanArgs sa;
-    sa.hist = reinterpret_cast<const int32_t*>(at(ws, pl.hist));
+    sa.group_hist = reinterpret_cast<int32_t*>(at(ws, kGroupHistOffset));
     sa.psum = with_stats ? reinterpret_cast<const double*>(at(ws, pl.psum)) : nullptr;
-    sa.chunk_base = reinterpret_cast<int32_t*>(at(ws, pl.base));
+    sa.group_base = reinterpret_cast<int32_t*>(at(ws, pl.gbase));
     sa.counts = counts;
     sa.offsets = offsets;
     sa.f = f;
     sa.p = p;
     sa.l_aux = l_aux;
     sa.psum_total = nullptr;
-    sa.nreal = nullptr;
+    sa.real_counter = nullptr;
     sa.shared_off = c->n_shared > 0 ? reinterpret_cast<int32_t*>(at(ws, pl.shared_off)) : nullptr;
     sa.T = c->T;
-    sa.nchunk = pl.nchunk;
+    sa.ngroups = pl.ngroups;
+    sa.npsum = pl.nchunk;
     sa.E = c->E;
     sa.k = c->k;
     sa.cap = (int)capacity_used(c);
@@ -278,17 +281,24 @@ moe_status_t run_router(const moe_config_t* c, const void* x, const void* w_rout
     a.hist = reinterpret_cast<int32_t*>(at(ws, pl.hist));
     a.psum = reinterpret_cast<double*>(at(ws, pl.psum));
     a.mask = mask;
-    a.nreal = reinterpret_cast<int32_t*>(at(ws, pl.nreal));
     a.T = c->T;
     a.d = c->d;
     a.E = c->E;
     a.k = c->k;
     a.nchunk = pl.nchunk;
+    a.group_chunks = pl.group_chunks;
+    a.ngroups = pl.ngroups;
+    a.psum_cap = pl.psum_cols;
     a.fuse_scan = fused != nullptr ? 1 : 0;
     a.counter = static_cast<unsigned int*>(ws) + kStatusCounterWord;
     if (fused != nullptr) {
+        // counters that only a fused scan reads and returns to zero
+        a.group_hist = reinterpret_cast<int32_t*>(at(ws, kGroupHistOffset));
         a.scan = *fused;
-        if (mask != nullptr) a.scan.nreal = a.nreal;  // statistics over the real tokens
+        if (mask != nullptr) {
+            a.real_counter = static_cast<int32_t*>(ws) + kStatusRealWord;
+            a.scan.real_counter = a.real_counter;  // statistics over the real tokens
+        }
     }
     a.st = status_of(ws);
     a.kernel = c->router_kernel;
@@ -300,7 +310,10 @@ moe_status_t run_scatter(const moe_config_t* c, const void* x, const int32_t* id
                          const int32_t* cap_e = nullptr) {
     ScatterArgs xa;
     xa.topk_idx = idx;
-    xa.chunk_base = reinterpret_cast<const int32_t*>(at(ws, pl.base));
+    xa.hist = reinterpret_cast<const int32_t*>(at(ws, pl.hist));
+    xa.group_base = reinterpret_cast<const int32_t*>(at(ws, pl.gbase));
+    xa.group_chunks = pl.group_chunks;
+    xa.ngroups = pl.ngroups;
     xa.offsets = offsets;
     xa.slot = slot;
     xa.src_assign = src_assign;
@@ -493,8 +506,9 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
         return MOE_ERR_INVALID_ARG;
     Plan pl;
     if ((st = check_ws(cfg, ws, ws_bytes, &pl)) != MOE_OK) return st;
-    if (launch_dispatch_hist(topk_idx, reinterpret_cast<int32_t*>(at(ws, pl.hist)), cfg->T, cfg->E, cfg->k, stream) !=
-        cudaSuccess)
+    if (launch_dispatch_hist(topk_idx, reinterpret_cast<int32_t*>(at(ws, pl.hist)),
+                             reinterpret_cast<int32_t*>(at(ws, kGroupHistOffset)), cfg->T, cfg->E, cfg->k,
+                             pl.group_chunks, pl.ngroups, stream) != cudaSuccess)
         return MOE_ERR_CUDA;
     const ScanArgs sa = scan_args(cfg, counts, offsets, nullptr, nullptr, nullptr, false, ws, pl);
     if (launch_dispatch_scan(sa, stream) != cudaSuccess) return MOE_ERR_CUDA;
@@ -806,7 +820,10 @@ moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int64_t T_global, const in
     if (cfg->T == 0) return MOE_OK;
     ScatterArgs xa;
     xa.topk_idx = o->topk_idx;
-    xa.chunk_base = reinterpret_cast<const int32_t*>(at(ws, pl.base));
+    xa.hist = reinterpret_cast<const int32_t*>(at(ws, pl.hist));
+    xa.group_base = reinterpret_cast<const int32_t*>(at(ws, pl.gbase));
+    xa.group_chunks = pl.group_chunks;
+    xa.ngroups = pl.ngroups;
     xa.offsets = dest_off;
     xa.slot = o->slot;
     xa.src_assign = nullptr;
@@ -957,7 +974,7 @@ moe_status_t moe_check_device_status(void* ws, size_t ws_bytes, cudaStream_t str
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
     if (site) *site = words[1];
     if (words[0] & (kErrTimeout | kErrRange)) {
-        if (cudaMemsetAsync(ws, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
         return (words[0] & kErrTimeout) ? MOE_ERR_TIMEOUT : MOE_ERR_RANGE;
     }

@@ -29,6 +29,7 @@
 
 #include "moe.h"
 #include "scan.cuh"
+#include "warp_mma.cuh"
 
 namespace moe {
 namespace {
@@ -46,27 +47,6 @@ __device__ __forceinline__ uint4 ldg_stream_128(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
-}
-
-__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Row position of slab row kk: rotated inside its 32-row block.
@@ -142,22 +122,24 @@ __device__ void router_finish(const RouterArgs& a, float* sL, int* sHist, bool a
             for (int e = 0; e < E; ++e) row[e] = 0.f;  // out of the probability sums
     }
     __syncthreads();
+    // per-chunk statistics: probability sums (psum columns are chunks here),
+    // expert counts, and the counts added into the chunk's group
     for (int i = tid; i < nchk * E; i += blockDim.x) {
         const int cl = i / E, e = i - cl * E;
         const int i0 = cl * kChunkTokens, i1 = min(ntok, i0 + kChunkTokens);
         double acc = 0.0;
         for (int r = i0; r < i1; ++r) acc += (double)sL[r * kLStride + e];
-        a.psum[(int64_t)e * a.nchunk + chunk0 + cl] = acc;
-        a.hist[(int64_t)e * a.nchunk + chunk0 + cl] = sHist[cl * kMaxExperts + e];
+        const int chunk = chunk0 + cl;
+        a.psum[(int64_t)e * a.nchunk + chunk] = acc;
+        const int n = sHist[cl * kMaxExperts + e];
+        a.hist[(int64_t)e * a.nchunk + chunk] = n;
+        if (n && a.group_hist) atomicAdd(a.group_hist + (int64_t)e * a.ngroups + chunk / a.group_chunks, n);
     }
-    if (a.mask != nullptr)
-        for (int cl = tid; cl < nchk; cl += blockDim.x) {
-            const int64_t c0 = t0 + (int64_t)cl * kChunkTokens;
-            const int64_t c1 = min64(c0 + kChunkTokens, a.T);
-            int n = 0;
-            for (int64_t t = c0; t < c1; ++t) n += a.mask[t] != 0;
-            a.nreal[chunk0 + cl] = n;
-        }
+    if (a.mask != nullptr && a.real_counter != nullptr && tid == 0) {
+        int n = 0;
+        for (int64_t t = t0; t < t0 + ntok; ++t) n += a.mask[t] != 0;
+        if (n) atomicAdd(a.real_counter, n);
+    }
     if (!a.fuse_scan) return;
     // last-CTA-done: the CTA that completes the arrival count runs the scan on
     // everyone's partials (fences order the partial stores before the count)
@@ -436,14 +418,19 @@ cudaError_t launch_f32_ep(RouterArgs a, cudaStream_t s) {
 }  // namespace
 
 // Router kernel choice: by the configuration only (never by T), so a token's
-// logits are the same whichever batch it is routed in.  The library's own
-// choice is the warp-MMA router; the tensor-core router on request.  Fed
-// logits (no GEMM to do) always take the warp router's softmax / top-k path.
+// logits are the same whichever batch it is routed in.  The library's choice
+// for bf16 is the warp-MMA router with the router weight resident across a
+// CTA cluster (same logits bit for bit as the slab-staged one, which takes the
+// shapes whose weight slices do not fit in shared memory); the tensor-core
+// router on request.  Fed logits (no GEMM) take the warp routers' selection.
 bool use_router_tc(const RouterArgs& a) { return a.kernel == MOE_ROUTER_TCGEN05 && router_tc_supported(a); }
 
-cudaError_t launch_router(const RouterArgs& a, bool bf16, cudaStream_t s) {
-    if (a.T == 0) return cudaSuccess;
+cudaError_t launch_router(const RouterArgs& a_in, bool bf16, cudaStream_t s) {
+    if (a_in.T == 0) return cudaSuccess;
+    RouterArgs a = a_in;
+    a.scan.npsum = a.nchunk;  // probability sums per chunk (the resident-weight router sets its own)
     if (bf16 && use_router_tc(a)) return launch_router_tc(a, a.st, s);
+    if (bf16 && a.kernel != MOE_ROUTER_WARP_MMA_STAGED && router_v2_supported(a)) return launch_router_v2(a, s);
     if (bf16) {
         switch ((a.E + 7) / 8) {
             case 1: return launch_bf16_nt<1>(a, s);

@@ -276,10 +276,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     if (lane == 0) {
                         a.psum[(int64_t)e * a.nchunk + chunk] = v;
                         a.hist[(int64_t)e * a.nchunk + chunk] = cnt;
+                        if (cnt && a.group_hist) atomicAdd(a.group_hist + (int64_t)e * a.ngroups + chunk / a.group_chunks, cnt);
                     }
                 }
                 const int nr = __popc(__ballot_sync(0xffffffffu, real));
-                if (a.mask != nullptr && lane == 0) a.nreal[chunk] = nr;
+                if (a.mask != nullptr && a.real_counter != nullptr && lane == 0 && nr) atomicAdd(a.real_counter, nr);
             }
         }
     }

@@ -1,16 +1,21 @@
 // Dispatch scan + load-balance statistics, as a block-level device function
-// shared by the standalone scan kernel and the router's last CTA.
+// shared by the standalone scan kernel and the routers' last CTA.
 //
-// For each expert e: exclusive scan of the per-chunk histogram over chunks
-// (the rank base of every chunk), the total n_e (counts, before the capacity
-// cut), and the sum of the per-chunk probability sums.  Then, in one thread,
-// the kept offsets offsets[e] = sum_{e'<e} min(n_e', cap) ("MoE: gating,
-// experts, load balancing, capacity factor" (dpshk.com/news/6005940) §2.4;
-// groups per expert as in "Hand-building a LLaMA4-MoE" (dpshk.com/news/
-// 5809432) §2.4) and f_e = n_e/(T*k), p_e = (1/T) sum_t p[t,e],
-// L_aux = alpha*E*sum_e f_e p_e (MoE-basics §2.3, §3.1), with T the number of
-// real tokens when padding is masked (LLaMA4-MoE §4.1).
-// Every sum has a fixed order, so results do not depend on scheduling.
+// For each expert e: exclusive scan of the per-group counts over groups (the
+// rank base of every group of chunks; the scatter adds the counts of the
+// earlier chunks inside the group), the total n_e (counts, before the
+// capacity cut), and the sum of the partial probability sums.  Then the kept
+// offsets offsets[e] = sum_{e'<e} min(n_e', cap) ("MoE: gating, experts, load
+// balancing, capacity factor" (dpshk.com/news/6005940) §2.4; groups per
+// expert as in "Hand-building a LLaMA4-MoE" (dpshk.com/news/5809432) §2.4)
+// and f_e = n_e/(T*k), p_e = (1/T) sum_t p[t,e], L_aux = alpha*E*sum_e f_e p_e
+// (MoE-basics §2.3, §3.1), with T the number of real tokens when padding is
+// masked (LLaMA4-MoE §4.1).
+//
+// The per-group counts were added with integer atomics (exact in any order);
+// every floating-point sum has a fixed order, so results do not depend on
+// scheduling.  The counters the producers accumulated (group counts, real
+// tokens) are returned to zero here for the next launch.
 #pragma once
 
 #include "internal.h"
@@ -26,102 +31,149 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
     return v;
 }
 
+// Copies n values global -> shared, eight loads in flight per thread.
+template <class T>
+__device__ __forceinline__ void stage_to_smem(T* dst, const T* src, int n) {
+    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+        T v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * blockDim.x;
+            v[u] = i < n ? __ldcg(src + i) : T(0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * blockDim.x;
+            if (i < n) dst[i] = v[u];
+        }
+    }
+}
+
 // All threads of the CTA call this; sCount / sP are shared arrays of kMaxExperts.
-// Partials are read with .cg loads (they may come from other CTAs of the same
-// grid); each lane first loads all of its chunks, so one round trip covers up
-// to 32 * kScanRegs chunks.
-constexpr int kScanRegs = 8;
-__device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, double* sP) {
+// Inputs written by other CTAs of the same grid are read with .cg loads.
+// With `scratch` (shared memory) large enough for the group counts and the
+// probability sums, every input is first copied there in a few round trips,
+// and the per-expert scans run from shared memory.
+__device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, double* sP, void* scratch = nullptr,
+                                           int scratch_bytes = 0) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
-    const int E = a.E, nc = a.nchunk;
+    // every argument in a register: no reloads from the parameter block after the stores
+    const int E = a.E, ng = a.ngroups, k = a.k, cap = a.cap;
+    const int64_t T = a.T;
+    const int npsum = a.psum != nullptr ? a.npsum : 0;
+    int32_t* __restrict__ group_hist = a.group_hist;
+    int32_t* __restrict__ group_base = a.group_base;
+    double* __restrict__ psum_total = a.psum_total;
+    int32_t* __restrict__ real_counter = a.real_counter;
+    const bool staged = scratch != nullptr && (int64_t)E * npsum * 8 + (int64_t)E * ng * 4 <= scratch_bytes;
+    const double* psum = a.psum;
+    const int32_t* ghist = group_hist;
+    if (staged) {
+        double* sPs = static_cast<double*>(scratch);
+        int32_t* sG = reinterpret_cast<int32_t*>(sPs + (int64_t)E * npsum);
+        stage_to_smem(sG, group_hist, E * ng);
+        if (npsum > 0) stage_to_smem(sPs, a.psum, E * npsum);
+        __syncthreads();
+        for (int i = tid; i < E * ng; i += blockDim.x) group_hist[i] = 0;
+        psum = sPs;
+        ghist = sG;
+    }
+    // a warp per expert: group bases and totals; the group counts go back to zero
     for (int e = warp; e < E; e += nwarps) {
-        const int32_t* h = a.hist + (int64_t)e * nc;
-        int32_t* cb = a.chunk_base + (int64_t)e * nc;
-        const double* pp = a.psum != nullptr ? a.psum + (int64_t)e * nc : nullptr;
+        const int32_t* gh = ghist + (int64_t)e * ng;
+        int32_t* gb = group_base + (int64_t)e * ng;
         int run = 0;
-        double ps = 0.0;
-        // lane owns chunks [c0 + lane*per, c0 + (lane+1)*per) of each 32*per span
-        for (int c0 = 0; c0 < nc; c0 += 32 * kScanRegs) {
-            const int per = min(kScanRegs, (nc - c0 + 31) / 32);
-            const int cbeg = c0 + lane * per;
-            int v[kScanRegs];
-            double q[kScanRegs];
-#pragma unroll
-            for (int i = 0; i < kScanRegs; ++i) {
-                const int c = cbeg + i;
-                const bool in = i < per && c < nc;
-                v[i] = in ? __ldcg(h + c) : 0;
-                q[i] = (in && pp != nullptr) ? __ldcg(pp + c) : 0.0;
-            }
-            int local = 0;
-#pragma unroll
-            for (int i = 0; i < kScanRegs; ++i) local += v[i];
-            const int incl = warp_inclusive_scan(local, lane);
-            int base = run + incl - local;
-#pragma unroll
-            for (int i = 0; i < kScanRegs; ++i) {
-                const int c = cbeg + i;
-                if (i < per && c < nc) cb[c] = base;
-                base += v[i];
-                ps += q[i];
+        for (int g0 = 0; g0 < ng; g0 += 32) {
+            const int g = g0 + lane;
+            const int v = g < ng ? (staged ? gh[g] : __ldcg(gh + g)) : 0;
+            const int incl = warp_inclusive_scan(v, lane);
+            if (g < ng) {
+                gb[g] = run + incl - v;
+                if (!staged) group_hist[(int64_t)e * ng + g] = 0;
             }
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
+        double ps = 0.0;
+        if (npsum > 0) {
+            // fixed order: lane-strided partial sums, then a fixed xor tree
+            const double* pp = psum + (int64_t)e * npsum;
+            for (int i = lane; i < npsum; i += 32) ps += staged ? pp[i] : __ldcg(pp + i);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        }
         if (lane == 0) {
             sCount[e] = run;
-            sP[e] = pp != nullptr ? ps : 0.0;  // divided by the real-token count below
-            if (a.psum_total != nullptr) a.psum_total[e] = ps;
+            sP[e] = ps;  // divided by the real-token count below
+            if (psum_total != nullptr) psum_total[e] = ps;
         }
     }
     __syncthreads();
     if (warp == 0) {
-        // real tokens: every token, or the per-chunk counts of unmasked tokens summed in chunk order
-        int64_t t_real = a.T;
-        if (a.nreal != nullptr) {
-            int64_t run = 0;
-            for (int c0 = 0; c0 < nc; c0 += 32) {
-                int v = c0 + lane < nc ? __ldcg(a.nreal + c0 + lane) : 0;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                run += v;
-            }
-            t_real = run;
-        }
-        if (lane == 0 && a.t_real_out != nullptr) a.t_real_out[0] = (int32_t)t_real;
-        if (lane == 0 && a.shared_off != nullptr) {
-            a.shared_off[0] = 0;
-            a.shared_off[1] = (int32_t)a.T;
+        int32_t* __restrict__ counts = a.counts;
+        int32_t* __restrict__ offsets = a.offsets;
+        float* __restrict__ fo = a.f;
+        float* __restrict__ po = a.p;
+        float* __restrict__ lo = a.l_aux;
+        int32_t* __restrict__ t_real_out = a.t_real_out;
+        int32_t* __restrict__ shared_off = a.shared_off;
+        const bool stats = a.psum != nullptr;
+        const float alpha = a.alpha;
+        // real tokens: every token, or the router's count of unmasked tokens
+        int64_t t_real = T;
+        if (real_counter != nullptr) t_real = __ldcg(real_counter);
+        __syncwarp();
+        if (lane == 0 && real_counter != nullptr) *real_counter = 0;
+        if (lane == 0 && t_real_out != nullptr) t_real_out[0] = (int32_t)t_real;
+        if (lane == 0 && shared_off != nullptr) {
+            shared_off[0] = 0;
+            shared_off[1] = (int32_t)T;
         }
         // kept offsets: exclusive scan of min(n_e, cap) over experts, 32 at a time
         int run = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
-            const int kept = e < E ? min(sCount[e], a.cap) : 0;
+            const int kept = e < E ? min(sCount[e], cap) : 0;
             const int incl = warp_inclusive_scan(kept, lane);
             if (e < E) {
-                a.counts[e] = sCount[e];
-                a.offsets[e] = run + incl - kept;
+                counts[e] = sCount[e];
+                offsets[e] = run + incl - kept;
             }
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) a.offsets[E] = run;
-        if (a.psum != nullptr) {
-            // statistics in a fixed order: lane-strided partial sums, then lane 0 adds them in lane order
+        if (lane == 0) offsets[E] = run;
+        if (stats) {
+            // statistics in a fixed order: lane-strided partial sums, then a fixed xor tree
             double l = 0.0;
             for (int e = lane; e < E; e += 32) {
-                const double f = t_real > 0 ? (double)sCount[e] / ((double)t_real * a.k) : 0.0;
+                const double f = t_real > 0 ? (double)sCount[e] / ((double)t_real * k) : 0.0;
                 const double pe = t_real > 0 ? sP[e] / (double)t_real : 0.0;
-                if (a.f) a.f[e] = (float)f;
-                if (a.p) a.p[e] = (float)pe;
+                if (fo) fo[e] = (float)f;
+                if (po) po[e] = (float)pe;
                 l += f * pe;
             }
-            double tot = 0.0;
-            for (int i = 0; i < 32; ++i) tot += __shfl_sync(0xffffffffu, l, i);
-            if (lane == 0 && a.l_aux) a.l_aux[0] = (float)((double)a.alpha * E * tot);
+            double tot = l;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            if (lane == 0 && lo) lo[0] = (float)((double)alpha * E * tot);
         }
     }
+}
+
+// The rank base of chunk `chunk` for expert e: its group's base plus the
+// chunk counts of the earlier chunks of the same group (integer sums, exact).
+__device__ __forceinline__ int chunk_base_of(const int32_t* __restrict__ hist, const int32_t* __restrict__ group_base,
+                                             int e, int chunk, int nchunk, int group_chunks, int ngroups) {
+    const int g = chunk / group_chunks;
+    int run = group_base[(int64_t)e * ngroups + g];
+    const int32_t* h = hist + (int64_t)e * nchunk;
+    int acc[4] = {0, 0, 0, 0};
+    int c = g * group_chunks;
+    for (; c + 4 <= chunk; c += 4) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += h[c + i];
+    }
+    for (; c < chunk; ++c) acc[0] += h[c];
+    return run + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
 }
 
 }  // namespace moe

@@ -96,11 +96,11 @@ def test_invalid_configs_rejected_on_host(lib):
     cfg = M.MoEConfig(T=8, d=128, ffn=128, E=4, k=2).c()
     cfg.dtype = 7
     assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
-    for rk in (-1, 3):
+    for rk in (-1, 4):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
         cfg.router_kernel = rk
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG
-    for name in ("auto", "warp_mma", "tcgen05"):
+    for name in ("auto", "warp_mma", "tcgen05", "warp_mma_staged"):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, router_kernel=name).c()
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
     for name in ("auto", "one_cta", "cta_pair"):

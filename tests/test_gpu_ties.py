@@ -14,9 +14,9 @@ Continuous random logits never tie, so these cases build ties on purpose:
     summation order.  The GPU's logits must then equal the oracle's bit for
     bit, and both sides decide on identical values without feeding anything.
 
-Both routers are covered: the warp-MMA kernel (every shape, fed or own
-logits) and the tcgen05 kernel (own logits, E % 8 == 0; it refuses fed
-logits).  Indices, counts, offsets, slots and src_assign are compared bit for
+All three routers are covered: the two warp-MMA kernels (resident weight and
+slab-staged; every shape, fed or own logits) and the tcgen05 kernel (own
+logits, E % 8 == 0; it refuses fed logits).  Indices, counts, offsets, slots and src_assign are compared bit for
 bit with the oracle, probabilities and weights within 1e-5 relative, and the
 layer output within the bf16 / fp32 output tolerance.
 """
@@ -119,7 +119,7 @@ TIE_CASES = [(4, "bf16", 300), (6, "bf16", 300), (8, "bf16", 1000), (64, "bf16",
 
 @pytest.mark.parametrize("E,dtype,T", TIE_CASES, ids=[f"E{e}-{dt}-T{t}" for e, dt, t in TIE_CASES])
 def test_router_ties_bit_exact(E, dtype, T):
-    routers = ["warp_mma"] + (["tcgen05"] if dtype == "bf16" and E % 8 == 0 else [])
+    routers = ["warp_mma", "warp_mma_staged"] + (["tcgen05"] if dtype == "bf16" and E % 8 == 0 else [])
     for k in range(1, min(E, 8) + 1):
         wl = W.Workload(f"ties_e{E}_k{k}", T=T, d=128, ffn=64, E=E, k=k, act="swiglu" if k % 2 else "gelu_bias",
                         dtype=dtype, capacity_factor=1.0, seed=300 + 10 * E + k)
@@ -136,13 +136,14 @@ def test_router_ties_bit_exact(E, dtype, T):
             cfg = M.MoEConfig.of(wl, router_kernel=router)
             _router_check(cfg, wl, inp, r_own, x, wd, exact_logits=True)
             _forward_check(cfg, wl, inp, r_own, x, wd)
-        # fed logits (warp router's selection path)
+        # fed logits (the warp routers' selection paths)
         L = tied_logits(T, E, k, seed=wl.seed + 1)
         r_fed = O.route(wl, inp, logits_feed=L)
         Ld = to_dev(L)
-        cfg = M.MoEConfig.of(wl, router_kernel="warp_mma")
-        _router_check(cfg, wl, inp, r_fed, x, wd, logits_in=Ld)
-        _forward_check(cfg, wl, inp, r_fed, x, wd, logits_in=Ld)
+        for router in ("warp_mma", "warp_mma_staged"):
+            cfg = M.MoEConfig.of(wl, router_kernel=router)
+            _router_check(cfg, wl, inp, r_fed, x, wd, logits_in=Ld)
+            _forward_check(cfg, wl, inp, r_fed, x, wd, logits_in=Ld)
         if "tcgen05" in routers:
             tc = M.MoEConfig.of(wl, router_kernel="tcgen05")
             with pytest.raises(M.MoEError) as e:
