@@ -384,6 +384,15 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
                 "achieved": round(achieved, 2), "peak": peak, "peak_source": f"{pk_src} ({'bf16 dense burst' if bound == 'tensor' else 'HBM copy'})",
                 "unit": unit, "frac": round(achieved / peak, 4),
                 "traffic": recorded_traffic(dname, name) if "gemm" in dname and wl.weights == "native" else None}
+    # the whole forward against HBM: every stage's algorithmic bytes (GEMMs: the
+    # weights of the experts hit plus their activation rows) over the step time;
+    # the bound that matters when the weights dominate (decode)
+    shared_bytes = wl.n_shared * ((nmat1 + 1) * wl.d * wl.ffn * bpe + 2 * wl.T * (wl.d + wl.ffn) * bpe)
+    fwd_bytes = algo["router"][1] + algo["scatter"][1] + gemm1_bytes + gemm2_bytes + shared_bytes + \
+        algo["combine"][1]
+    fwd_gbs = fwd_bytes / (total_ms / steps / 1e3) / 1e9
+    forward_roofline = {"bound": "hbm", "bytes_per_step": int(fwd_bytes), "achieved": round(fwd_gbs, 1),
+                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(fwd_gbs / pk["hbm_gbs"], 4)}
     stages = {}
     for j, n in enumerate(names):
         b, w = algo[n]
@@ -477,7 +486,7 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
                    "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
                    "launch": "timed steps replayed from one captured CUDA graph",
                    "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel, "dispatch": a.dispatch},
-        "roofline": roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * steps,
+        "roofline": roofline, "forward_roofline": forward_roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * steps,
         "clocks": clocks, "cpu_baseline": cpu,
     }
     del layer, weights, x, flush, evict, graph
@@ -487,7 +496,7 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
 
 def per_config_entry(line: dict) -> dict:
     """The summary of one workload's line kept in the headline's per_config table."""
-    keep = ("value", "unit", "ms_per_step", "steps", "dtype", "roofline", "stages", "clocks")
+    keep = ("value", "unit", "ms_per_step", "steps", "dtype", "roofline", "forward_roofline", "stages", "clocks")
     ent = {k: line[k] for k in keep}
     ent["rows_dispatched"] = line["config"]["rows_dispatched"]
     ent["e2e"] = {k: line["e2e"][k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")}

@@ -134,6 +134,24 @@ typedef enum { MOE_DISPATCH_AUTO = 0, MOE_DISPATCH_COPY = 1, MOE_DISPATCH_GATHER
  *                       FFNs stream.  Shared experts keep native weights. */
 typedef enum { MOE_WEIGHTS_NATIVE = 0, MOE_WEIGHTS_INT8 = 1 } moe_weight_format_t;
 
+/* Where moe_forward and moe_dp_finish apply the routing weights topk_w.
+ *   MOE_WEIGHTING_AUTO      the library's choice: EPILOGUE where it applies
+ *                           (bf16 with native weights), else COMBINE;
+ *   MOE_WEIGHTING_COMBINE   y_perm holds each expert's output rounded to the
+ *                           dtype, and the combine forms sum_j w[t,j] y(t,j)
+ *                           in fp32;
+ *   MOE_WEIGHTING_EPILOGUE  bf16 with native weights: the second expert GEMM
+ *                           multiplies each fp32 output row (after b2) by its
+ *                           routing weight before its one rounding to bf16
+ *                           ("Loop-MoE" §2.1 / MoE-basics §4.4: the weighted
+ *                           expert output is formed per row), and the combine
+ *                           is a plain fp32 sum of the k weighted rows.  The
+ *                           other dtypes and INT8 weights fall back to COMBINE.
+ * The two orders round differently (last bits of out); both are within the
+ * layer's bf16 tolerance.  The expert-parallel calls and moe_combine always
+ * weight in the combine. */
+typedef enum { MOE_WEIGHTING_AUTO = 0, MOE_WEIGHTING_COMBINE = 1, MOE_WEIGHTING_EPILOGUE = 2 } moe_weighting_t;
+
 /* Layer shape.  Limits: 0 <= T, T*k < 2^31; 1 <= E <= 64; 1 <= k <= min(E, 8).
  * bf16: d % 64 == 0 and ffn % 64 == 0.  f32: d % 4 == 0 and ffn % 4 == 0. */
 typedef struct {
@@ -151,6 +169,7 @@ typedef struct {
     int32_t dispatch;          /* moe_dispatch_mode_t (0: library's choice) */
     int32_t n_shared;          /* shared experts, 0..8 (LLaMA4-MoE §5.2; see moe_forward) */
     int32_t weight_format;     /* moe_weight_format_t of the routed experts */
+    int32_t weighting;         /* moe_weighting_t (0: library's choice) */
 } moe_config_t;
 
 /* Expert and router parameters (device, config dtype unless stated). */
@@ -302,7 +321,9 @@ moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const
  *   n_shared > 0: the shared experts (weights->shared_*) run on every token,
  *     padding included, and out[t] = sum_j w[t,j] y(t,j) + sum_s y_s(t),
  *     accumulated in fp32 (routed terms first, then shared experts in order)
- *     and rounded once. */
+ *     and rounded once.
+ *   cfg->weighting: whether w[t,j] y(t,j) is formed in the second GEMM's
+ *     epilogue (rounded there) or in the combine (moe_weighting_t). */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
                          const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs, void* ws,
                          size_t ws_bytes, cudaStream_t stream);

@@ -33,6 +33,8 @@ MOE_GEMM_AUTO, MOE_GEMM_ONE_CTA, MOE_GEMM_CTA_PAIR = 0, 1, 2
 GEMM_KERNELS = {"auto": MOE_GEMM_AUTO, "one_cta": MOE_GEMM_ONE_CTA, "cta_pair": MOE_GEMM_CTA_PAIR}
 MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER = 0, 1, 2
 DISPATCH_MODES = {"auto": MOE_DISPATCH_AUTO, "copy": MOE_DISPATCH_COPY, "gather": MOE_DISPATCH_GATHER}
+MOE_WEIGHTING_AUTO, MOE_WEIGHTING_COMBINE, MOE_WEIGHTING_EPILOGUE = 0, 1, 2
+WEIGHTINGS = {"auto": MOE_WEIGHTING_AUTO, "combine": MOE_WEIGHTING_COMBINE, "epilogue": MOE_WEIGHTING_EPILOGUE}
 
 
 class MoEError(RuntimeError):
@@ -46,7 +48,7 @@ class MoEConfigC(ctypes.Structure):
                 ("k", ctypes.c_int32), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("aux_alpha", ctypes.c_float), ("router_kernel", ctypes.c_int32),
                 ("gemm_kernel", ctypes.c_int32), ("dispatch", ctypes.c_int32), ("n_shared", ctypes.c_int32),
-                ("weight_format", ctypes.c_int32)]
+                ("weight_format", ctypes.c_int32), ("weighting", ctypes.c_int32)]
 
 
 class MoEWeightsC(ctypes.Structure):
@@ -135,6 +137,7 @@ class MoEConfig:
     dispatch: str = "auto"       # "auto" | "copy" | "gather"
     n_shared: int = 0            # shared experts, applied to every token with weight 1
     weights: str = "native"      # routed experts' weights: "native" (the dtype) or "int8" (codes + scales)
+    weighting: str = "auto"      # routing weights applied in: "auto" | "combine" | "epilogue" (second GEMM)
 
     def c(self) -> MoEConfigC:
         return MoEConfigC(self.T, self.d, self.ffn, self.E, self.k,
@@ -142,7 +145,7 @@ class MoEConfig:
                           MOE_ACT_SWIGLU if self.act == "swiglu" else MOE_ACT_GELU_BIAS,
                           float(self.capacity_factor), float(self.aux_alpha), ROUTER_KERNELS[self.router_kernel],
                           GEMM_KERNELS[self.gemm_kernel], DISPATCH_MODES[self.dispatch], int(self.n_shared),
-                          1 if self.weights == "int8" else 0)
+                          1 if self.weights == "int8" else 0, WEIGHTINGS[self.weighting])
 
     @property
     def torch_dtype(self) -> torch.dtype:

@@ -6,8 +6,10 @@
 // balancing, capacity factor" (dpshk.com/news/6005940) §3.1), over the kept
 // assignments only, fp32 accumulation in ascending j, then plus each shared
 // expert's output (LLaMA4-MoE §5.2: fixed experts in every token's
-// computation), rounded once.  One warp per token, 16-byte vector loads of
-// the expert rows, no atomics.
+// computation), rounded once.  Without weights (topk_w null) the expert rows
+// were already multiplied by their routing weights in the second GEMM's
+// epilogue and the combine is their plain sum.  One warp per token, 16-byte
+// vector loads of the expert rows, no atomics.
 //
 // Statistics: f_e = n_e / (T*k), p_e = mean_t softmax[t,e],
 // L_aux = alpha * E * sum_e f_e p_e (MoE-basics §2.3 and §3.1).
@@ -19,9 +21,8 @@ namespace {
 // EP: the expert rows are read from the output buffer of the rank holding
 // each expert (peer memory over NVLink), so the gather back to token order is
 // this step's all-to-all, fused with the weighted sum.
-template <bool BF16, bool EP>
-__global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
-    constexpr int U = 4;               // 16-byte vectors per lane per expert row (x2 rows in flight)
+template <bool BF16, bool EP, int U>  // U: 16-byte vectors per lane per expert row (x2 rows in flight)
+__global__ void __launch_bounds__(256, 8 / U) combine_kernel(CombineArgs a) {
     constexpr int VEC = BF16 ? 8 : 4;  // elements per 16-byte vector
     const int warps_per_cta = blockDim.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
         [[maybe_unused]] const uint4* y_l = Y;
         if (lane < a.k) {
             s_l = a.slot[t * a.k + lane];
-            w_l = a.topk_w[t * a.k + lane];
+            w_l = a.topk_w != nullptr ? a.topk_w[t * a.k + lane] : 1.0f;
             if constexpr (EP) {
                 if (s_l >= 0) {
                     const int e = a.topk_idx[t * a.k + lane];
@@ -213,22 +214,30 @@ __global__ void selftest_wait_kernel(DevStatus st) {
     }
 }
 
-}  // namespace
-
-cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s) {
-    if (a.T == 0) return cudaSuccess;
-    const int64_t blocks = min64((a.T + 7) / 8, (int64_t)sm_count() * 8);
+template <int U>
+void launch_combine_u(const CombineArgs& a, bool bf16, int64_t blocks, cudaStream_t s) {
     const bool ep = a.e_per_rank > 0;
     if (bf16 && ep)
-        combine_kernel<true, true><<<(unsigned)blocks, 256, 0, s>>>(a);
+        combine_kernel<true, true, U><<<(unsigned)blocks, 256, 0, s>>>(a);
     else if (bf16)
-        combine_kernel<true, false><<<(unsigned)blocks, 256, 0, s>>>(a);
+        combine_kernel<true, false, U><<<(unsigned)blocks, 256, 0, s>>>(a);
     else if (ep)
-        combine_kernel<false, true><<<(unsigned)blocks, 256, 0, s>>>(a);
+        combine_kernel<false, true, U><<<(unsigned)blocks, 256, 0, s>>>(a);
     else
-        combine_kernel<false, false><<<(unsigned)blocks, 256, 0, s>>>(a);
+        combine_kernel<false, false, U><<<(unsigned)blocks, 256, 0, s>>>(a);
+}
+
+}  // namespace
+
+// Rows in passes of 128 16-byte vectors (4 per lane, both rows of an expert
+// pair in flight), two CTAs per SM.  (Whole 2048-wide rows per pass, 8
+// vectors per lane, were measured slower: half the warps fit per SM.)
+cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s) {
+    if (a.T == 0) return cudaSuccess;
+    launch_combine_u<4>(a, bf16, min64((a.T + 7) / 8, (int64_t)sm_count() * 8), s);
     return cudaGetLastError();
 }
+
 
 cudaError_t launch_aux_from_probs(const int32_t* counts, const float* probs, float* f, float* p, float* l_aux,
                                   int64_t T, int E, int k, float alpha, cudaStream_t s) {

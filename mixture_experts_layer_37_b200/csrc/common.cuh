@@ -133,6 +133,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, uin
         : "memory");
 }
 
+// Four rows of a 2-D tensor into consecutive rows of this CTA's shared
+// memory (tile::gather4: the map's box is one row high; c0 is the innermost
+// coordinate, r0..r3 the rows); completion counted on `bar` as transaction
+// bytes.  No multicast.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* map, uint64_t* bar, int32_t c0, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared (L2 only), and an arrival on
 // `bar` once all of this thread's earlier cp.async copies have landed (the
 // arrival counts toward the barrier's expected count: .noinc).

@@ -49,17 +49,20 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
     scan_block(a, sCount, sP);
 }
 
-// One CTA per chunk of kChunkTokens tokens (<= 256 assignments): ranks,
-// capacity test, slot and src_assign, then the row copies x[t] -> x_perm[slot]
-// (each warp copies two rows at a time with 16-byte vectors).  Under expert
-// parallelism the destination is the receive buffer of the expert's rank, so
-// the copies are this step's all-to-all: stores into peer memory over NVLink.
-__global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a) {
+// `nsplit` CTAs per chunk of kChunkTokens tokens (<= 256 assignments): each
+// computes the chunk's ranks, capacity test and slots (the first one writes
+// slot and src_assign), then copies its share of the rows x[t] -> x_perm[slot]
+// (each warp copies two rows at a time with 16-byte vectors; splitting a
+// chunk's copies over several CTAs keeps every SM busy when chunks are few).
+// Under expert parallelism the destination is the receive buffer of the
+// expert's rank, so the copies are this step's all-to-all: stores into peer
+// memory over NVLink.
+__global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a, int nsplit) {
     __shared__ int sWarpBase[kScatterWarps][kMaxExperts];
     __shared__ uint4* sDst[kScatterThreads];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, k = a.k;
-    const int chunk = blockIdx.x;
+    const int chunk = blockIdx.x / nsplit, part = blockIdx.x - chunk * nsplit;
     const int64_t t0 = (int64_t)chunk * kChunkTokens;
     const int ntok = (int)min64(kChunkTokens, a.T - t0);
     const int nA = ntok * k;
@@ -93,12 +96,12 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
             if (a.row_limit > 0 && (s < 0 || s >= a.row_limit)) {
                 if (a.st.word != nullptr) report_range(a.st, SITE_EP_SCATTER_ROW);
                 s = -1;
-            } else if (a.src_assign != nullptr) {
+            } else if (a.src_assign != nullptr && part == 0) {
                 a.src_assign[s] = (int32_t)(a_base + tid);
             }
         }
     }
-    if (tid < nA) a.slot[a_base + tid] = s;
+    if (tid < nA && part == 0) a.slot[a_base + tid] = s;
     const bool ep = a.e_per_rank > 0;
     if (a.x_perm == nullptr && !ep) return;  // rows gathered by the first GEMM instead
     uint4* dst = nullptr;
@@ -112,12 +115,13 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
     // 16 loads in flight per lane); dropped assignments copy nothing
     const int vecs = a.row_bytes / 16;
     const uint4* X = static_cast<const uint4*>(a.x);
-    for (int q = warp; q < nA; q += 2 * kScatterWarps) {
+    const int qb = part * nA / nsplit, qe = (part + 1) * nA / nsplit;  // this CTA's assignments
+    for (int q = qb + warp; q < qe; q += 2 * kScatterWarps) {
         const int q1 = q + kScatterWarps;
         uint4* d0 = sDst[q];
-        uint4* d1 = q1 < nA ? sDst[q1] : nullptr;
+        uint4* d1 = q1 < qe ? sDst[q1] : nullptr;
         const uint4* src0 = X + ((a_base + q) / k) * vecs;
-        const uint4* src1 = X + ((a_base + (q1 < nA ? q1 : q)) / k) * vecs;
+        const uint4* src1 = X + ((a_base + (q1 < qe ? q1 : q)) / k) * vecs;
         for (int v0 = lane; v0 < vecs; v0 += 32 * 8) {
             uint4 b0[8], b1[8];
 #pragma unroll
@@ -305,7 +309,11 @@ cudaError_t launch_dispatch_scan(const ScanArgs& a, cudaStream_t s) {
 
 cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s) {
     if (a.nchunk == 0) return cudaSuccess;
-    scatter_kernel<<<a.nchunk, kScatterThreads, 0, s>>>(a);
+    // with row copies to do and fewer than two chunks per SM, each chunk's copies go to several CTAs
+    int nsplit = 1;
+    const bool copies = a.x_perm != nullptr || a.e_per_rank > 0;
+    while (copies && nsplit < 4 && (int64_t)a.nchunk * nsplit < 2 * (int64_t)sm_count()) nsplit *= 2;
+    scatter_kernel<<<(unsigned)(a.nchunk * nsplit), kScatterThreads, 0, s>>>(a, nsplit);
     return cudaGetLastError();
 }
 

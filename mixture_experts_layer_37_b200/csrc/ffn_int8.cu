@@ -10,19 +10,20 @@
 //
 // The FFN kernel is built for decode-sized batches, where an expert holds a
 // handful of rows and the layer time is the time to stream the weights.  One
-// CTA per (expert, 256-column tile), 288 threads:
-//   warp 0, lane 0   producer: per stage one TMA tile of codes [64 K x 256
+// CTA per (expert, 128-column tile), two CTAs per SM, 288 threads:
+//   warp 0, lane 0   producer: per stage one TMA tile of codes [64 K x 128
 //                    columns] (two for SwiGLU: gate and up) and one of the
 //                    expert's activations [4 rows x 64 K], 4 stages;
-//   warps 1-8        each takes 8 of a stage's 64 K rows for all 256 columns
-//                    (8 per lane: one 8-byte load of codes per K row), only
-//                    as many activation rows as the pass holds (up to 4),
-//                    fp32 FMAs; the eight partial sums are added in warp order
-//                    and the scale (and bias / activation) applied once per
-//                    output.
-// On B200 the codes' conversion to fp32 bounds this kernel (issue-bound at
-// about 3 TB/s of codes on the decode workload), so it matches the bf16
-// tensor-core path's time while streaming half the bytes.
+//   warps 1-8        each takes 8 of a stage's 64 K rows for all 128 columns
+//                    (4 per lane: one 4-byte load of codes per K row), only
+//                    as many activation rows as the pass holds (up to 4);
+//                    codes become fp32 by a byte permute and one packed
+//                    subtraction per two codes, and the FMAs run two at a
+//                    time (f32x2, each rounded as a scalar fmaf); the eight
+//                    partial sums are added in warp order and the scale (and
+//                    bias / activation) applied once per output.
+// 128-column tiles give the decode workload's ~57 busy experts 16 tiles each,
+// about 6 per SM: the last partial wave costs little.
 // Weight bytes per element: 1 instead of 2.  An expert with more than 4 rows
 // streams its weights once per 4 rows (correct, slow for large batches).
 // Every wait is bounded in time, as in the other kernels.
@@ -35,14 +36,14 @@ namespace {
 
 constexpr int kQThreads = 288;             // producer warp + 8 consumer warps
 constexpr int kQWarps = 8;                  // consumer warps: each takes 8 of a stage's 64 K rows
-constexpr int kQCols = 256;                 // output columns per CTA (8 per consumer lane)
+constexpr int kQCols = 128;                 // output columns per CTA (4 per consumer lane)
 constexpr int kQKB = 64;                    // K rows per stage
 constexpr int kQRows = 4;                   // expert rows per pass
 constexpr int kQStages = 4;
-constexpr int kQWTile = kQKB * kQCols;      // 16 KB of codes
+constexpr int kQWTile = kQKB * kQCols;      // 8 KB of codes
 constexpr int kQXTile = kQRows * kQKB * 2;  // 512 B of bf16 activations
 constexpr int kQStage = 2 * kQWTile + kQXTile;
-constexpr int kQRed = kQWarps * kQRows * kQCols * 2 * 4;  // partial sums of the 8 warps (64 KB)
+constexpr int kQRed = kQWarps * kQRows * kQCols * 2 * 4;  // partial sums of the 8 warps (32 KB)
 constexpr int kQSmem = kQStages * kQStage + kQRed + 256 + 128;
 
 enum { Q_SWIGLU = 0, Q_GELU = 1, Q_PLAIN = 2, Q_PLAIN_BIAS = 3 };
@@ -87,65 +88,85 @@ struct QArgs {
 __device__ __forceinline__ float silu_q(float x) { return x / (1.0f + __expf(-x)); }
 __device__ __forceinline__ float gelu_q(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// Four int8 codes (one 32-bit word) to exact floats without the integer
-// conversion unit: with the sign bit flipped a code b becomes the unsigned
-// byte u = b + 128; placed as the low mantissa byte of 2^23 (bit pattern
-// 0x4B0000uu) it reads as 2^23 + u, and subtracting 2^23 + 128 leaves b.
-__device__ __forceinline__ void codes_to_float(uint32_t word, float* f) {
-    const uint32_t u = word ^ 0x80808080u;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t bits;
-        // bytes of {0x4B000000 : u}: result = [u.byte j, 0x00, 0x00, 0x4B]
-        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(bits) : "r"(u), "r"(0x4B000000u), "r"(0x7540u | (uint32_t)j));
-        f[j] = __uint_as_float(bits) - 8388736.0f;
-    }
+// Packed pairs of fp32 values (the f32x2 arithmetic of sm_100: two independent
+// fp32 operations per instruction, each rounded as its scalar form).
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
 }
 
-// One consumer warp's share of a stage: K rows [16w, 16w+16), all 256
-// columns (8 per lane), the first RT activation rows.
+// Four int8 codes (one 32-bit word) to exact floats, as two packed pairs,
+// without the integer conversion unit: with the sign bit flipped a code b
+// becomes the unsigned byte u = b + 128; placed as the low mantissa byte of
+// 2^23 (bit pattern 0x4B0000uu) it reads as 2^23 + u, and subtracting
+// 2^23 + 128 leaves b exactly.
+__device__ __forceinline__ void codes_to_pairs(uint32_t word, uint64_t* f) {
+    const uint32_t u = word ^ 0x80808080u;
+    uint32_t bits[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        // bytes of {0x4B000000 : u}: result = [u.byte j, 0x00, 0x00, 0x4B]
+        asm("prmt.b32 %0, %1, %2, %3;" : "=r"(bits[j]) : "r"(u), "r"(0x4B000000u), "r"(0x7540u | (uint32_t)j));
+    const uint32_t m = __float_as_uint(8388736.0f);
+    const uint64_t magic = pack2(m, m);
+    f[0] = sub2(pack2(bits[0], bits[1]), magic);
+    f[1] = sub2(pack2(bits[2], bits[3]), magic);
+}
+
+// One consumer warp's share of a stage: K rows [8w, 8w+8), all 128 columns
+// (4 per lane, as two packed pairs), the first RT activation rows.
 template <bool TWO, int RT>
-__device__ __forceinline__ void consume_stage(const uint8_t* st, int w, int lane, float (&acc0)[kQRows][8],
-                                              float (&acc1)[kQRows][8]) {
-    const uint2* w0 = reinterpret_cast<const uint2*>(st) + lane;
-    const uint2* w1 = reinterpret_cast<const uint2*>(st + kQWTile) + lane;
+__device__ __forceinline__ void consume_stage(const uint8_t* st, int w, int lane, uint64_t (&acc0)[kQRows][2],
+                                              uint64_t (&acc1)[kQRows][2]) {
+    const uint32_t* w0 = reinterpret_cast<const uint32_t*>(st) + lane;
+    const uint32_t* w1 = reinterpret_cast<const uint32_t*>(st + kQWTile) + lane;
     const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + 2 * kQWTile);
 #pragma unroll 4
     for (int i = 0; i < kQKB / kQWarps; ++i) {
         const int kk = w * (kQKB / kQWarps) + i;
-        const uint2 q0 = w0[kk * (kQCols / 8)];
-        uint2 q1 = make_uint2(0, 0);
-        if (TWO) q1 = w1[kk * (kQCols / 8)];
-        float c0[8], c1[8];
-        codes_to_float(q0.x, c0);
-        codes_to_float(q0.y, c0 + 4);
-        if (TWO) {
-            codes_to_float(q1.x, c1);
-            codes_to_float(q1.y, c1 + 4);
-        }
+        const uint32_t q0 = w0[kk * (kQCols / 4)];
+        const uint32_t q1 = TWO ? w1[kk * (kQCols / 4)] : 0u;
+        uint64_t c0[2], c1[2];
+        codes_to_pairs(q0, c0);
+        if (TWO) codes_to_pairs(q1, c1);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const float xv = __bfloat162float(xs[r * kQKB + kk]);
+            const uint32_t xb = __float_as_uint(__bfloat162float(xs[r * kQKB + kk]));
+            const uint64_t xv = pack2(xb, xb);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                acc0[r][j] = fmaf(xv, c0[j], acc0[r][j]);
-                if (TWO) acc1[r][j] = fmaf(xv, c1[j], acc1[r][j]);
+            for (int j = 0; j < 2; ++j) {
+                acc0[r][j] = fma2(xv, c0[j], acc0[r][j]);
+                if (TWO) acc1[r][j] = fma2(xv, c1[j], acc1[r][j]);
             }
         }
     }
 }
 
-// tmQ0/tmQ1: codes as a 2-D uint8 tensor [E*K, N], box [64 rows, 256 columns];
+// tmQ0/tmQ1: codes as a 2-D uint8 tensor [E*K, N], box [64 rows, 128 columns];
 // tmA: activations [rows, K] bf16, box [4 rows, 64 K].
 template <int MODE>
-__global__ void __launch_bounds__(kQThreads, 1) ffn_int8_kernel(const __grid_constant__ CUtensorMap tmQ0,
+__global__ void __launch_bounds__(kQThreads, 2) ffn_int8_kernel(const __grid_constant__ CUtensorMap tmQ0,
                                                                const __grid_constant__ CUtensorMap tmQ1,
                                                                const __grid_constant__ CUtensorMap tmA, QArgs p) {
     constexpr bool TWO = MODE == Q_SWIGLU;
     constexpr uint32_t kBytes = (TWO ? 2 : 1) * kQWTile + kQXTile;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
-    float* red = reinterpret_cast<float*>(smem + kQStages * kQStage);  // [warp][2][row][256]
+    float* red = reinterpret_cast<float*>(smem + kQStages * kQStage);  // [warp][2][row][kQCols]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kQStage + kQRed);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
@@ -208,11 +229,11 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_int8_kernel(const __grid_con
         bool ok = true;  // the same in all four warps: set from the shared abort flag after each barrier
         for (int r0 = row_begin; r0 < row_end && ok; r0 += kQRows) {
             const int nr = min(kQRows, row_end - r0);
-            float acc0[kQRows][8], acc1[kQRows][8];
+            uint64_t acc0[kQRows][2], acc1[kQRows][2];
 #pragma unroll
             for (int r = 0; r < kQRows; ++r)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc0[r][j] = acc1[r][j] = 0.f;
+                for (int j = 0; j < 2; ++j) acc0[r][j] = acc1[r][j] = 0ull;  // +0.0f pairs
             for (int kb = 0; kb < kblocks; ++kb) {
                 if (__shfl_sync(0xffffffffu, *abort_flag, 0)) { ok = false; break; }
                 const bool got = mbar_wait_bounded(&full[stage], phase, tmo);
@@ -240,9 +261,13 @@ __global__ void __launch_bounds__(kQThreads, 1) ffn_int8_kernel(const __grid_con
             if (ok) {
                 for (int r = 0; r < nr; ++r)
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        red[((w * 2 + 0) * kQRows + r) * kQCols + 8 * lane + j] = acc0[r][j];
-                        if (TWO) red[((w * 2 + 1) * kQRows + r) * kQCols + 8 * lane + j] = acc1[r][j];
+                    for (int j = 0; j < 2; ++j) {
+                        float* d0 = red + ((w * 2 + 0) * kQRows + r) * kQCols + 4 * lane + 2 * j;
+                        unpack2(acc0[r][j], d0[0], d0[1]);
+                        if (TWO) {
+                            float* d1 = red + ((w * 2 + 1) * kQRows + r) * kQCols + 4 * lane + 2 * j;
+                            unpack2(acc1[r][j], d1[0], d1[1]);
+                        }
                     }
             }
             named_barrier_sync(1, kQWarps * 32);

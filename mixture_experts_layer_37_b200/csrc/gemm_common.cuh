@@ -51,6 +51,9 @@ struct GemmParams {
     const __nv_bfloat16* gx = nullptr;    // [T, K] or null (A read through its tensor map)
     const int32_t* src_assign = nullptr;  // [R]
     int k = 0;
+    // routing weights of the output rows (second GEMM): row s is multiplied by
+    // row_w[src_assign[s]] in fp32, after the bias, before the one rounding; or null
+    const float* row_w = nullptr;         // [T*k]
 };
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
@@ -90,12 +93,19 @@ __device__ __forceinline__ void decode_tile(int tile, const int* mt_prefix, cons
     rows = min(bm, s_off[e + 1] - row0);
 }
 
+// The routing weight of output row `row` (1 without row weights or for a row
+// that is not stored).
+__device__ __forceinline__ float row_weight(const GemmParams& p, int row, bool valid) {
+    return p.row_w != nullptr && valid ? __ldg(p.row_w + __ldg(p.src_assign + row)) : 1.0f;
+}
+
 // Epilogue of one warp for one tile: its 32 accumulator rows (TMEM lanes of
-// `tbase`), activation, one rounding to bf16, and the store of the rows that
+// `tbase`), activation (or bias, times the row's routing weight `rw` when the
+// GEMM has row weights), one rounding to bf16, and the store of the rows that
 // are valid.  `wb` is the warp's 256-entry bias staging row.  Warp-collective.
 template <int MODE>
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tbase, __nv_bfloat16* orow, bool valid,
-                                              int n0, int e, __nv_bfloat16* wb, int lane) {
+                                              int n0, int e, __nv_bfloat16* wb, int lane, float rw = 1.0f) {
     if (MODE == MODE_SWIGLU) {
         for (int c = 0; c < 128; c += 16) {
             uint32_t g[16], u[16];
@@ -146,6 +156,10 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tbas
                 if (MODE == MODE_GELU) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) x[i] = gelu_f(x[i]);
+                }
+                if (p.row_w != nullptr) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] *= rw;
                 }
                 uint32_t pk[8];
 #pragma unroll

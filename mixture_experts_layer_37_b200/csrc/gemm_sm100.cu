@@ -47,9 +47,8 @@ constexpr int kStages = 4;
 constexpr int kAStageBytes = BM * BK * 2;                  // 16 KB
 constexpr int kBStageBytes = 4 * kBBoxBytes;               // 32 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;   // 48 KB
-constexpr int kTokBytes = BM * 4;                          // gathered tile: token of each row
 constexpr int kSmemBytes =
-    kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + kTokBytes + 1024 /*alignment*/;
+    kStages * kStageBytes + 1024 /*barriers + tables*/ + kBiasBytes + 1024 /*alignment*/;
 constexpr uint32_t kIdesc = make_idesc(BM, BN_MMA);
 constexpr uint32_t kIdesc64 = make_idesc(BM / 2, BN_MMA);
 
@@ -72,14 +71,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* mt_prefix = reinterpret_cast<int*>(tmem_slot + 2);   // [E+1]
     int* s_off = mt_prefix + (kMaxExperts + 1);                // [E+1]
     __nv_bfloat16* s_bias = reinterpret_cast<__nv_bfloat16*>(smem + kStages * kStageBytes + 1024);  // [4][256]
-    int* s_tok = reinterpret_cast<int*>(smem + kStages * kStageBytes + 1024 + kBiasBytes);           // [BM]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            // gathered A: the 32 producer lanes' cp.async arrivals join the TMA's
-            mbar_init(&full[s], GATHER ? 33 : 1);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&tfull[0], 1);
@@ -113,59 +110,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (warp == 0 && GATHER) {
-        // ------------------------------------------------ gathering producer (whole warp)
-        // A tile: lane L copies 16-byte chunk L % 8 of rows L / 8 + 4i of the
-        // tile straight from the token rows (8 lanes read one row's 128 bytes),
-        // to the place the 128-byte swizzle gives it; B as in the TMA producer.
+        // ------------------------------------------------ gathering producer
+        // A tile: 32 TMA gathers of four token rows each (tile::gather4 over
+        // the token activations, a one-row box of 64 columns, 128-byte
+        // swizzle), lane l copying tile rows 4l..4l+3 into their place in the
+        // swizzled tile, all lanes issuing at once; lane 0 arms the stage and
+        // loads B as the plain producer does.
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued_mask = 0, issued_par = 0;
         bool stop = false;
         const int R = s_off[p.E];
-        const int ch = lane & 7;
         for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
             int e, row0, rows, nt;
             decode_tile(tile, mt_prefix, s_off, p.n_tiles, BM, e, row0, rows, nt);
             const int n0 = nt * p.bn_out;
-            __syncwarp();  // every lane is done with the previous tile's tokens
-            for (int r = lane; r < BM; r += 32) {
-                const int row = row0 + r;
-                s_tok[r] = row < R ? p.src_assign[row] / p.k : 0;  // rows past R: any valid row, masked later
-            }
-            __syncwarp();
-            for (int kb = 0; kb < kblocks; ++kb) {
-                if (__shfl_sync(0xffffffffu, *abort_flag, 0)) { stop = true; break; }
-                const bool free_ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, tmo);
-                if (!__all_sync(0xffffffffu, free_ok)) {
-                    if (lane == 0) give_up(SITE_GEMM_PRODUCER_EMPTY);
-                    stop = true;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[stage], kBStageBytes);
-                    uint8_t* b_dst = sB + stage * kBStageBytes;
-                    const int krow = e * p.K + kb * BK;
-                    if (MODE == MODE_SWIGLU) {
-                        tma_load_2d(b_dst, &tmB0, &full[stage], n0, krow);
-                        tma_load_2d(b_dst + kBBoxBytes, &tmB0, &full[stage], n0 + 64, krow);
-                        tma_load_2d(b_dst + 2 * kBBoxBytes, &tmB1, &full[stage], n0, krow);
-                        tma_load_2d(b_dst + 3 * kBBoxBytes, &tmB1, &full[stage], n0 + 64, krow);
-                    } else {
+            int tok[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            tma_load_2d(b_dst + i * kBBoxBytes, &tmB0, &full[stage], n0 + 64 * i, krow);
+            for (int i = 0; i < 4; ++i) {
+                const int row = row0 + 4 * lane + i;
+                tok[i] = row < R ? p.src_assign[row] / p.k : 0;  // rows past R: any valid row, masked later
+            }
+            for (int kb = 0; kb < kblocks; ++kb) {
+                if (lane == 0) {
+                    if (*abort_flag) {
+                        stop = true;
+                    } else if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, tmo)) {
+                        give_up(SITE_GEMM_PRODUCER_EMPTY);
+                        stop = true;
+                    } else {
+                        mbar_arrive_expect_tx(&full[stage], kStageBytes);
+                        uint8_t* b_dst = sB + stage * kBStageBytes;
+                        const int krow = e * p.K + kb * BK;
+                        if (MODE == MODE_SWIGLU) {
+                            tma_load_2d(b_dst, &tmB0, &full[stage], n0, krow);
+                            tma_load_2d(b_dst + kBBoxBytes, &tmB0, &full[stage], n0 + 64, krow);
+                            tma_load_2d(b_dst + 2 * kBBoxBytes, &tmB1, &full[stage], n0, krow);
+                            tma_load_2d(b_dst + 3 * kBBoxBytes, &tmB1, &full[stage], n0 + 64, krow);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                tma_load_2d(b_dst + i * kBBoxBytes, &tmB0, &full[stage], n0 + 64 * i, krow);
+                        }
+                        issued_mask |= 1u << stage;
+                        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     }
                 }
-                uint8_t* a_dst = sA + stage * kAStageBytes;
-                const __nv_bfloat16* gsrc = p.gx + kb * BK + ch * 8;
-#pragma unroll 8
-                for (int i = 0; i < BM / 4; ++i) {
-                    const int r = (lane >> 3) + 4 * i;
-                    cp_async_16_cg(a_dst + r * 128 + ((ch ^ (r & 7)) << 4), gsrc + (int64_t)s_tok[r] * p.K);
-                }
-                cp_async_mbar_arrive_noinc(&full[stage]);
-                issued_mask |= 1u << stage;
-                issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                // the stage is armed (or the producer stops) before any lane's copy
+                stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+                if (stop) break;
+                tma_gather4(sA + stage * kAStageBytes + lane * 4 * 128, &tmA, &full[stage], kb * BK, tok[0], tok[1],
+                            tok[2], tok[3]);
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -249,8 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    // gathered A was written by cp.async (generic proxy); the MMA reads it through the async proxy
-                    if (GATHER) fence_proxy_async_smem();
                     const uint32_t a_addr = smem_u32(sA + stage * kAStageBytes);
                     const uint32_t b_addr = smem_u32(sB + stage * kBStageBytes);
 #pragma unroll
@@ -301,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = r < rows && (!m64 || lane < 16);
             __nv_bfloat16* orow = p.out + (int64_t)(row0 + (valid ? r : 0)) * p.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
-            epilogue_rows<MODE>(p, tbase, orow, valid, nt * p.bn_out, e, wb, lane);
+            epilogue_rows<MODE>(p, tbase, orow, valid, nt * p.bn_out, e, wb, lane, row_weight(p, row0 + r, valid));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -408,9 +401,12 @@ cudaError_t launch_one(int mode, bool pair, const CUtensorMap& a, const CUtensor
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     if (a.rows_cap <= 0) return cudaSuccess;
     const bool swiglu = a.act == 0;
-    // A maps use 128-row boxes (one CTA's half of a pair tile, or a whole single-CTA tile)
+    // A maps use 128-row boxes (one CTA's half of a pair tile, or a whole single-CTA tile); a first
+    // GEMM gathering its rows reads the token activations through a one-row box (tile::gather4)
     CUtensorMap mA1, mB1, mB1u, mA2, mB2;
-    bool ok = make_map(&mA1, a.x_perm, (uint64_t)a.d, (uint64_t)a.rows_cap, (uint64_t)a.d * 2, 64, 128);
+    bool ok = a.gather_x != nullptr
+                  ? make_map(&mA1, a.gather_x, (uint64_t)a.d, (uint64_t)a.gather_rows, (uint64_t)a.d * 2, 64, 1)
+                  : make_map(&mA1, a.x_perm, (uint64_t)a.d, (uint64_t)a.rows_cap, (uint64_t)a.d * 2, 64, 128);
     ok = ok && make_map(&mB1, a.w1, (uint64_t)a.ffn, (uint64_t)a.E * a.d, (uint64_t)a.ffn * 2, 64, BK);
     if (swiglu)
         ok = ok && make_map(&mB1u, a.w_up, (uint64_t)a.ffn, (uint64_t)a.E * a.d, (uint64_t)a.ffn * 2, 64, BK);
@@ -451,7 +447,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p2.n_tiles = (a.d + 255) / 256;
     p2.st = a.st;
     p2.gx = nullptr;
-    p2.src_assign = nullptr;
+    p2.src_assign = a.row_w != nullptr ? a.src_assign : nullptr;
+    p2.row_w = a.row_w;
     p2.k = a.k;
     return launch_one(MODE_PLAIN, pair2, mA2, mB2, mB2, p2, a.rows_cap, s);
 }

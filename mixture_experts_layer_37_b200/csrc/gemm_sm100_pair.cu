@@ -48,10 +48,12 @@ constexpr uint32_t kIdescPHalf = make_idesc(BMP / 2, BN_MMA);
 // Epilogue of one warp for `ncols` accumulator columns starting at TMEM column
 // offset 0 of `tbase`, written to output columns [out0, out0 + ncols) (SwiGLU:
 // ncols/2 outputs from [gate 64 | up 64] groups).  `wb` is the warp's bias
-// staging row.  Warp-collective.
+// staging row; `rw` the row's routing weight (GEMMs with row weights).
+// Warp-collective.
 template <int MODE>
 __device__ __forceinline__ void epilogue_pair(const GemmParams& p, uint32_t tbase, __nv_bfloat16* orow, bool valid,
-                                              int out0, int ncols, int e, __nv_bfloat16* wb, int lane) {
+                                              int out0, int ncols, int e, __nv_bfloat16* wb, int lane,
+                                              float rw = 1.0f) {
     if (MODE == MODE_SWIGLU) {
         for (int g = 0; g < ncols; g += 128) {
             const int o = out0 + g / 2;
@@ -106,6 +108,10 @@ __device__ __forceinline__ void epilogue_pair(const GemmParams& p, uint32_t tbas
                 if (MODE == MODE_GELU) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) x[i] = gelu_f(x[i]);
+                }
+                if (p.row_w != nullptr) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] *= rw;
                 }
                 uint32_t pk[8];
 #pragma unroll
@@ -304,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool valid = r < rows;
             __nv_bfloat16* orow = p.out + (int64_t)(row0 + (valid ? r : 0)) * p.N;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MMA);
-            epilogue_pair<MODE>(p, tbase, orow, valid, out0, ncols, e, wb, lane);
+            epilogue_pair<MODE>(p, tbase, orow, valid, out0, ncols, e, wb, lane, row_weight(p, row0 + r, valid));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * acc);

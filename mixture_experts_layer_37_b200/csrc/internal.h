@@ -161,7 +161,7 @@ cudaError_t launch_ep_prepare(const EpPrepareArgs& a, cudaStream_t s);
 struct CombineArgs {
     const void* y_perm = nullptr;    // [R_max, d]
     const int32_t* slot = nullptr;   // [T, k]
-    const float* topk_w = nullptr;   // [T, k]
+    const float* topk_w = nullptr;   // [T, k], or null: rows already weighted (plain sum)
     void* out = nullptr;             // [T, d]
     const void* y_shared = nullptr;  // [n_shared, T, d] shared experts' outputs, added with weight 1, or null
     int n_shared = 0;
@@ -199,9 +199,13 @@ struct FfnArgs {
     int gemm_kernel = 0;         // moe_gemm_kernel_t
     // when gather_x != null the first GEMM reads its rows straight from the
     // tokens (row s = token src_assign[s] / k) and x_perm is not used
-    const void* gather_x = nullptr;    // [T, d] or null
+    const void* gather_x = nullptr;    // [gather_rows, d] or null
     const int32_t* src_assign = nullptr;
+    int64_t gather_rows = 0;           // T: rows of gather_x
     int k = 0;
+    // bf16 only: when row_w != null the second GEMM multiplies output row s by
+    // row_w[src_assign[s]] (its routing weight) before rounding
+    const float* row_w = nullptr;      // [T*k] or null
     // INT8 weights (w1 / w_up / w2 hold codes): per-expert, per-output-column scales
     bool int8 = false;
     const float* w1_scale = nullptr;   // [E, ffn]

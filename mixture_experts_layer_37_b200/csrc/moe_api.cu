@@ -48,7 +48,8 @@ moe_status_t check_config(const moe_config_t* c) {
     if (isnan(c->capacity_factor) || isnan(c->aux_alpha) || c->router_kernel < MOE_ROUTER_AUTO ||
         c->router_kernel > MOE_ROUTER_WARP_MMA_STAGED || c->gemm_kernel < MOE_GEMM_AUTO || c->gemm_kernel > MOE_GEMM_CTA_PAIR ||
         c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER || c->n_shared < 0 ||
-        c->weight_format < MOE_WEIGHTS_NATIVE || c->weight_format > MOE_WEIGHTS_INT8)
+        c->weight_format < MOE_WEIGHTS_NATIVE || c->weight_format > MOE_WEIGHTS_INT8 ||
+        c->weighting < MOE_WEIGHTING_AUTO || c->weighting > MOE_WEIGHTING_EPILOGUE)
         return MOE_ERR_INVALID_ARG;
     if (c->n_shared > kMaxShared) return MOE_ERR_UNSUPPORTED;
     if (c->weight_format == MOE_WEIGHTS_INT8 && c->dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED;
@@ -335,9 +336,16 @@ bool gathers(const moe_config_t* c) {
     return c->dtype == MOE_DT_BF16 && c->dispatch == MOE_DISPATCH_GATHER && c->weight_format == MOE_WEIGHTS_NATIVE;
 }
 
+// Whether moe_forward / moe_dp_finish weight the expert rows in the second
+// GEMM's epilogue (then the combine is a plain sum of the k rows).
+bool weights_in_epilogue(const moe_config_t* c) {
+    return c->dtype == MOE_DT_BF16 && c->weight_format == MOE_WEIGHTS_NATIVE && c->weighting != MOE_WEIGHTING_COMBINE;
+}
+
 moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* x_perm, const int32_t* offsets,
                      void* y_perm, void* ws, const Plan& pl, cudaStream_t s, cudaEvent_t between = nullptr,
-                     const void* gather_x = nullptr, const int32_t* src_assign = nullptr) {
+                     const void* gather_x = nullptr, const int32_t* src_assign = nullptr,
+                     const float* row_w = nullptr) {
     FfnArgs f;
     f.act = c->act;
     f.E = c->E;
@@ -358,7 +366,11 @@ moe_status_t run_ffn(const moe_config_t* c, const moe_weights_t* w, const void* 
     f.gemm_kernel = c->gemm_kernel;
     f.gather_x = gather_x;
     f.src_assign = src_assign;
+    f.gather_rows = c->T;
     f.k = c->k;
+    f.row_w = row_w;
+    if ((row_w != nullptr || gather_x != nullptr) && src_assign == nullptr) return MOE_ERR_INVALID_ARG;
+    if (row_w != nullptr && !weights_in_epilogue(c)) return MOE_ERR_INVALID_ARG;
     if (c->weight_format == MOE_WEIGHTS_INT8) {
         // INT8 routed experts: rows always come from the sorted copy
         if (x_perm == nullptr) return MOE_ERR_INVALID_ARG;
@@ -584,6 +596,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
     const bool gather = gathers(cfg);
+    const bool weighted = weights_in_epilogue(cfg);
     {
         const NvtxRange r("moe_forward/scatter");
         st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
@@ -594,7 +607,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     {
         const NvtxRange r("moe_forward/expert_ffn");
         st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, ev ? ev[n++] : nullptr,
-                     gather ? x : nullptr, o->src_assign);
+                     gather ? x : nullptr, o->src_assign, weighted ? o->topk_w : nullptr);
     }
     if (st != MOE_OK) return st;
     if (!mark()) return MOE_ERR_CUDA;
@@ -604,7 +617,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     }
     {
         const NvtxRange r("moe_forward/combine");
-        st = run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
+        st = run_combine(cfg, y_perm, o->slot, weighted ? nullptr : o->topk_w, o->out, stream,
                          cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
     }
     if (st != MOE_OK) return st;
@@ -724,11 +737,12 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
     void* x_perm = at(ws, pl.xperm);
     void* y_perm = at(ws, pl.yperm);
     const bool gather = gathers(cfg);
+    const bool weighted = weights_in_epilogue(cfg);
     st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
                      stream, dp.cap_e);
     if (st != MOE_OK) return st;
     st = run_ffn(cfg, weights, x_perm, o->offsets, y_perm, ws, pl, stream, nullptr, gather ? x : nullptr,
-                 o->src_assign);
+                 o->src_assign, weighted ? o->topk_w : nullptr);
     if (st != MOE_OK) return st;
     if (cfg->n_shared > 0) {
         // the shared experts' row offsets {0, T} were written by the prepare kernel
@@ -736,7 +750,7 @@ moe_status_t moe_dp_finish(const moe_config_t* cfg, int64_t T_global, const int3
         int n = 0;
         if ((st = run_shared(cfg, weights, x, ws, pl, stream, nomark, nullptr, &n)) != MOE_OK) return st;
     }
-    return run_combine(cfg, y_perm, o->slot, o->topk_w, o->out, stream,
+    return run_combine(cfg, y_perm, o->slot, weighted ? nullptr : o->topk_w, o->out, stream,
                        cfg->n_shared > 0 ? at(ws, pl.ys) : nullptr);
 }
 

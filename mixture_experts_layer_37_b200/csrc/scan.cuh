@@ -160,20 +160,21 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
 }
 
 // The rank base of chunk `chunk` for expert e: its group's base plus the
-// chunk counts of the earlier chunks of the same group (integer sums, exact).
+// chunk counts of the earlier chunks of the same group (integer sums, exact),
+// read 32 at a time with every load of a batch in flight together.
 __device__ __forceinline__ int chunk_base_of(const int32_t* __restrict__ hist, const int32_t* __restrict__ group_base,
                                              int e, int chunk, int nchunk, int group_chunks, int ngroups) {
     const int g = chunk / group_chunks;
     int run = group_base[(int64_t)e * ngroups + g];
     const int32_t* h = hist + (int64_t)e * nchunk;
-    int acc[4] = {0, 0, 0, 0};
-    int c = g * group_chunks;
-    for (; c + 4 <= chunk; c += 4) {
+    for (int c0 = g * group_chunks; c0 < chunk; c0 += 32) {
+        int v[32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += h[c + i];
+        for (int i = 0; i < 32; ++i) v[i] = c0 + i < chunk ? h[c0 + i] : 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) run += v[i];
     }
-    for (; c < chunk; ++c) acc[0] += h[c];
-    return run + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    return run;
 }
 
 }  // namespace moe

@@ -41,8 +41,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_config_struct_layout_matches_header():
-    assert ctypes.sizeof(M.MoEConfigC) == 64
+    assert ctypes.sizeof(M.MoEConfigC) == 72
     assert M.MoEConfigC.capacity_factor.offset == 32 and M.MoEConfigC.n_shared.offset == 56
+    assert M.MoEConfigC.weighting.offset == 64
     assert ctypes.sizeof(M.MoEWeightsC) == 15 * 8 and ctypes.sizeof(M.MoEOutputsC) == 12 * 8
 
 
@@ -109,6 +110,9 @@ def test_invalid_configs_rejected_on_host(lib):
     for name in ("auto", "copy", "gather"):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, dispatch=name).c()
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
+    for name in ("auto", "combine", "epilogue"):
+        cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, weighting=name).c()
+        assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_OK
     assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, n_shared=8).c()),
                                   ctypes.byref(size)) == M.MOE_OK
     assert lib.moe_workspace_size(ctypes.byref(M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2, n_shared=9).c()),
@@ -119,7 +123,7 @@ def test_invalid_configs_rejected_on_host(lib):
                                                            weights="int8").c()), ctypes.byref(size)) == \
         M.MOE_ERR_UNSUPPORTED
     for field, v in (("gemm_kernel", 3), ("gemm_kernel", -1), ("dispatch", 3), ("dispatch", -1), ("n_shared", -1),
-                     ("weight_format", 2), ("weight_format", -1)):
+                     ("weight_format", 2), ("weight_format", -1), ("weighting", 3), ("weighting", -1)):
         cfg = M.MoEConfig(T=8, d=128, ffn=128, E=8, k=2).c()
         setattr(cfg, field, v)
         assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(size)) == M.MOE_ERR_INVALID_ARG

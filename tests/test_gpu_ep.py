@@ -14,6 +14,7 @@ ExpertParallelMoE with CUDA IPC mappings of each other's buffers and host
 barriers (gloo), and a refusal test feeds counts and slots that do not match
 the routing and checks that the kernels refuse the rows (MOE_ERR_RANGE)
 instead of touching memory outside the buffers."""
+import dataclasses
 import os
 import socket
 
@@ -100,6 +101,12 @@ def run_emulated(wl, bounds, wd, x, all_counts_fn=None, fill=None, mask=None):
     return ranks
 
 
+def _whole_cfg(wl):
+    """The one-device forward the expert-parallel calls must equal bit for bit:
+    they weight the expert rows in the combine, so this one does too."""
+    return dataclasses.replace(M.MoEConfig.of(wl), weighting="combine")
+
+
 def _device_weights(wl, inp):
     wd = weights_dev(wl, inp)
     if wl.weights == "int8":
@@ -113,7 +120,7 @@ def test_ep_equals_whole_batch(wl, bounds):
     wd = _device_weights(wl, inp)
     x = to_dev(inp["x"])
     mask = mask_dev(inp)
-    whole = M.MoELayer(M.MoEConfig.of(wl), wd).forward(x, token_mask=mask)
+    whole = M.MoELayer(_whole_cfg(wl), wd).forward(x, token_mask=mask)
     torch.cuda.synchronize()
     world = len(bounds) - 1
     El = wl.E // world
@@ -280,7 +287,7 @@ def test_ep_two_processes_over_ipc():
     inp = W.make_inputs(wl)
     wd = weights_dev(wl, inp)
     x = to_dev(inp["x"])
-    whole = M.MoELayer(M.MoEConfig.of(wl), wd).forward(x)
+    whole = M.MoELayer(_whole_cfg(wl), wd).forward(x)
     torch.cuda.synchronize()
     bounds = [0, 420, 1000]
     ctx = mp.get_context("spawn")

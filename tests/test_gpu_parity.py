@@ -5,6 +5,8 @@ span several tiles, ragged tails, drops, k = E, E = 1, T = 1 and fp32.
 Inputs come from the seeded generator; expected values come only from the
 oracle.  Where both sides must take a discrete decision on identical values
 (top-k, capacity ranks), the oracle's fp32 logits are fed to both."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -185,6 +187,20 @@ def _check_workload(wl, full_size: bool, router: str = "auto", gemm: str = "auto
     ok, e_, s_ = out_close(got, ref["out"], wl.dtype)
     assert ok, f"layer output max err {e_} vs scale {s_}"
     first = {n: v.clone() for n, v in o.items()}
+
+    # ---- 7b. bf16 with native weights: the forward weights each expert row in the
+    #          second GEMM's epilogue; with the weights applied in the combine
+    #          instead, routing is the same bit for bit and the output is within
+    #          the same tolerance (only the rounding order differs)
+    if wl.dtype == "bf16" and wl.weights == "native":
+        lc = M.MoELayer(dataclasses.replace(cfg_feed, weighting="combine"), wd)
+        oc = lc.forward(x, logits_in=dev(feed), token_mask=tm)
+        lc.check()
+        for n in ("topk_idx", "topk_w", "counts", "offsets", "slot", "f", "p", "l_aux"):
+            assert torch.equal(oc[n].cpu(), o[n].cpu()), f"{n} depends on the weighting order"
+        ok, e_, s_ = out_close(host_f64(oc["out"])[toks], ref["out"], wl.dtype)
+        assert ok, f"layer output (weights in the combine) max err {e_} vs scale {s_}"
+        del lc, oc
 
     # ---- 8. determinism: a second run is bit-identical
     o2 = layer_feed.forward(x, logits_in=dev(feed), token_mask=tm)
