@@ -112,16 +112,19 @@ typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_ONE_CTA = 1, MOE_GEMM_CTA_PAIR = 2 } 
 
 /* How the first expert GEMM of moe_forward / moe_dp_finish gets its rows
  * (bf16; the f32 path always copies).  Same results bit for bit.
- *   MOE_DISPATCH_AUTO    the library's choice (currently COPY: the gathering
- *                        producer's 16-byte copies keep the tensor cores
- *                        waiting, so its first GEMM is slower than copy plus
- *                        TMA tiles);
+ *   MOE_DISPATCH_AUTO    the library's choice (currently COPY: the gathered
+ *                        tiles take 32 TMA gathers of four 128-byte rows per
+ *                        16 KB stage, which the TMA unit issues about 3x
+ *                        slower than the tensor cores consume them, so the
+ *                        gathering first GEMM is slower than copy plus TMA
+ *                        tiles on B200);
  *   MOE_DISPATCH_COPY    the dispatch kernel copies each kept row to the
  *                        expert-sorted x_perm, which the GEMM reads by TMA;
  *   MOE_DISPATCH_GATHER  the GEMM's producer warp gathers the token rows of x
- *                        straight into its shared-memory tiles (one-CTA
- *                        kernel); the dispatch kernel writes only slot and
- *                        src_assign, and x_perm is never written. */
+ *                        straight into its shared-memory tiles with TMA
+ *                        tile::gather4 (one-CTA kernel); the dispatch kernel
+ *                        writes only slot and src_assign, and x_perm is never
+ *                        written. */
 typedef enum { MOE_DISPATCH_AUTO = 0, MOE_DISPATCH_COPY = 1, MOE_DISPATCH_GATHER = 2 } moe_dispatch_mode_t;
 
 /* Storage of the routed experts' weights.

@@ -37,10 +37,12 @@
 // Exchange buffers are guarded by mbarriers with cluster-scope release and
 // acquire (full: every writer lane has stored; empty: the finisher has read),
 // so the producer keeps streaming the next tile while the finishers work.
-// Finish (ranks 0 and 1, one chunk each per tile): eight lanes per token,
-// shuffle reductions inside each lane group, outputs, and the chunk's
-// statistics; probability sums accumulate per CTA in a fixed order.  The last
-// CTA runs the dispatch scan with its shared memory as scratch.
+//   warps 9-16 (ranks 0 and 1) finish one 32-token chunk each per tile, while
+//             the consumer warps already run the next tile's products: eight
+//             lanes per token, shuffle reductions inside each lane group,
+//             outputs, and the chunk's statistics; probability sums
+//             accumulate per CTA in a fixed order.
+// The last CTA runs the dispatch scan with its shared memory as scratch.
 // Every wait is bounded in time; on expiry the kernel records the site, skips
 // the remaining work, keeps every barrier count, and returns.
 #include <math.h>
@@ -57,8 +59,11 @@
 namespace moe {
 namespace {
 
-constexpr int kQW = 8;                        // consumer warps
-constexpr int kV2Threads = (kQW + 1) * 32;    // + the TMA producer warp
+constexpr int kQW = 8;                        // consumer warps, and finisher warps
+constexpr int kProducerWarp = kQW;            // the TMA producer
+constexpr int kFinWarp0 = kQW + 1;            // first finisher warp
+constexpr int kV2Threads = (2 * kQW + 1) * 32;
+constexpr int kConsumerBar = 1, kFinisherBar = 2;  // named barriers of the two warp groups
 constexpr int kTile = 64;                     // tokens per tile: four 16-token m-tiles, two chunks
 constexpr int kStageBytes = kTile * 128;      // one 64-column block pair of a tile
 constexpr int kMinStages = 4, kMaxStages = 16;
@@ -130,7 +135,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-// Finish of one 32-token chunk by the 8 consumer warps (all of them call it;
+// Finish of one 32-token chunk by the 8 finisher warps (all of them call it;
 // `work` false skips the work but keeps the three barriers).  Eight lanes per
 // token: warp w takes tokens 4w..4w+3, lane group g = lane/8 one token, lane
 // j = lane%8 of the group the experts j, j+8, ..., so every reduction over a
@@ -146,13 +151,14 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // chunk's statistics: probability sums per expert in a fixed order (fp64),
 // expert counts (per-lane counters, no atomics), and the counts added into
 // the chunk's group.
+// `ft` is the thread's index in the finisher group (0..255).
 template <int M, class Release>  // M = experts per lane = ceil(E / 8)
 __device__ __forceinline__ void finish_chunk(const RouterArgs& a, int chunk, const float* xb, int xs, const float* sBias,
-                                             float* sPc, int* sH, double* sPsum, int* sReal, bool work,
+                                             float* sPc, int* sH, double* sPsum, int* sReal, bool work, int ft,
                                              Release release) {
     const int PS = xs;  // row stride of the statistics scratch, as of the exchange buffer
     constexpr int NONE = 0x7fffffff;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = ft >> 5, lane = ft & 31;
     const int grp = lane >> 3, jl = lane & 7;
     // every argument in a register: no reloads from the parameter block after the stores
     const int E = a.E, k = a.k, nchunk = a.nchunk, ngroups = a.ngroups, gchunks = a.group_chunks;
@@ -186,7 +192,7 @@ __device__ __forceinline__ void finish_chunk(const RouterArgs& a, int chunk, con
         }
         v[m] = x;
     }
-    named_barrier_sync(1, kQW * 32);
+    named_barrier_sync(kFinisherBar, kQW * 32);
     release();  // every warp has read the exchange buffer
     int cnt[M];
 #pragma unroll
@@ -283,7 +289,7 @@ __device__ __forceinline__ void finish_chunk(const RouterArgs& a, int chunk, con
         const unsigned nreal = __popc(__ballot_sync(0xffffffffu, real && jl == 0));
         if (lane == 0) atomicAdd(sReal, (int)nreal);
     }
-    named_barrier_sync(1, kQW * 32);
+    named_barrier_sync(kFinisherBar, kQW * 32);
     if (work && warp == 0) {
         for (int e = lane; e < E; e += 32) {
             // the chunk's probability sum in a fixed order: four interleaved token chains, then pairwise
@@ -301,7 +307,7 @@ __device__ __forceinline__ void finish_chunk(const RouterArgs& a, int chunk, con
             if (n && ghist) atomicAdd(ghist + (int64_t)e * ngroups + chunk / gchunks, n);
         }
     }
-    named_barrier_sync(1, kQW * 32);
+    named_barrier_sync(kFinisherBar, kQW * 32);
 }
 
 template <int NTL, int M>
@@ -365,7 +371,7 @@ __global__ void __launch_bounds__(kV2Threads, 1)
         *abort_flag = 1;
     };
 
-    if (warp == kQW) {
+    if (warp == kProducerWarp) {
         if (lane == 0 && !fed) {
             // ------------------------------------------------ TMA producer (starts before the weights land)
             int stage = 0;
@@ -396,7 +402,7 @@ __global__ void __launch_bounds__(kV2Threads, 1)
         }
         __syncwarp();
         cluster_wait();
-    } else {
+    } else if (warp < kQW) {
         // ---------------------------------------------------- consumers
         if (!fed) {
             // the resident weight: W_r rows of the CTA's blocks (4j + 2pr + {0,1}), its experts
@@ -423,7 +429,7 @@ __global__ void __launch_bounds__(kV2Threads, 1)
             cp_async_commit();
             cp_async_wait_all();
         }
-        named_barrier_sync(1, kQW * 32);
+        named_barrier_sync(kConsumerBar, kQW * 32);
         cluster_wait();  // every CTA's barriers exist before any remote arrival
 
         const int u = warp & 1, mt = warp >> 1;
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(kV2Threads, 1)
         const int s_part = 2 * pr + u;
         const int lt0 = 16 * (mt & 1) + rg, lt1 = lt0 + 8;  // token rows inside the chunk
         int stage = 0;
-        uint32_t phase = 0, xe_par = 0, xf_par = 0;
+        uint32_t phase = 0, xe_par = 0;
         bool dead = false;
         for (int tile = cid; tile < ntiles; tile += ncl) {
             dead = dead || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
@@ -503,8 +509,18 @@ __global__ void __launch_bounds__(kV2Threads, 1)
                 }
                 xe_par ^= 1u;
             }
-            if (finisher) {
-                // the 8 consumer warps finish this CTA's chunk of the tile
+        }
+    } else {
+        // ---------------------------------------------------- finishers (ranks 0 and 1)
+        // warps kFinWarp0.. finish this CTA's chunk of each tile while the
+        // consumers already run the next tile's products
+        cluster_wait();  // every CTA's barriers exist before any remote arrival (the releases)
+        const int ft = (int)threadIdx.x - kFinWarp0 * 32;
+        uint32_t xf_par = 0;
+        bool dead = false;
+        if (finisher) {
+            for (int tile = cid; tile < ntiles; tile += ncl) {
+                dead = dead || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
                 if (!fed && !dead) {
                     const bool ok = mbar_wait_cluster_bounded(xfull, xf_par, tmo);
                     if (!__all_sync(0xffffffffu, ok)) {
@@ -515,15 +531,17 @@ __global__ void __launch_bounds__(kV2Threads, 1)
                 xf_par ^= 1u;
                 const int chunk = tile * 2 + rank;
                 // the exchange buffer is free again for every writer of the cluster
-                // (lane r of warp 0 signals CTA r: one release each, in parallel)
+                // (finisher thread r signals CTA r: one release each, in parallel)
                 auto release = [&]() {
-                    if (!fed && (int)threadIdx.x < cs)
-                        mbar_arrive_cluster(mapa_shared(smem_u32(&xempty[rank]), threadIdx.x));
+                    if (!fed && ft < cs) mbar_arrive_cluster(mapa_shared(smem_u32(&xempty[rank]), (uint32_t)ft));
                 };
                 finish_chunk<M>(a, chunk, xbuf, xs, a.bias != nullptr ? sBias : nullptr, sPc, sH, sPsum,
-                                  &sMisc[2], !dead && chunk < nchunk, release);
+                                &sMisc[2], !dead && chunk < nchunk, ft, release);
             }
         }
+    }
+    __syncthreads();
+    {
         // this CTA's probability sums (zero when it finished no chunk) and real-token count
         if (warp == 0) {
             for (int e = lane; e < E; e += 32) a.psum[(int64_t)e * gridDim.x + blockIdx.x] = sPsum[e];
@@ -531,7 +549,6 @@ __global__ void __launch_bounds__(kV2Threads, 1)
                 atomicAdd(a.real_counter, sMisc[2]);
         }
     }
-    __syncthreads();
     cluster_sync_all();  // no CTA leaves while a peer may still store into it or arrive on its barriers
     if (!a.fuse_scan) return;
     // last CTA to finish runs the scan on everyone's statistics (its ring and weight slice as scratch)

@@ -53,10 +53,14 @@ __device__ __forceinline__ void stage_to_smem(T* dst, const T* src, int n) {
 // Inputs written by other CTAs of the same grid are read with .cg loads.
 // With `scratch` (shared memory) large enough for the group counts and the
 // probability sums, every input is first copied there in a few round trips,
-// and the per-expert scans run from shared memory.
+// and the per-expert work reads shared memory.  The experts are handled side by
+// side: P threads per expert (the largest power of two with P*E threads in the
+// block, at most 32) sum the expert's probability-sum columns (thread j takes
+// columns j, j+P, ..., then a fixed xor tree over the P threads), and the first
+// of them scans the expert's groups in order.
 __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, double* sP, void* scratch = nullptr,
                                            int scratch_bytes = 0) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthreads = blockDim.x;
     // every argument in a register: no reloads from the parameter block after the stores
     const int E = a.E, ng = a.ngroups, k = a.k, cap = a.cap;
     const int64_t T = a.T;
@@ -74,38 +78,41 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
         stage_to_smem(sG, group_hist, E * ng);
         if (npsum > 0) stage_to_smem(sPs, a.psum, E * npsum);
         __syncthreads();
-        for (int i = tid; i < E * ng; i += blockDim.x) group_hist[i] = 0;
+        for (int i = tid; i < E * ng; i += nthreads) group_hist[i] = 0;
         psum = sPs;
         ghist = sG;
     }
-    // a warp per expert: group bases and totals; the group counts go back to zero
-    for (int e = warp; e < E; e += nwarps) {
-        const int32_t* gh = ghist + (int64_t)e * ng;
-        int32_t* gb = group_base + (int64_t)e * ng;
+    int P = 32;
+    while (P > 1 && P * E > nthreads) P >>= 1;
+    const int ex = tid / P, jx = tid - (tid / P) * P;  // this thread's expert and its place in the expert's group
+    double ps = 0.0;
+    if (ex < E && npsum > 0) {
+        const double* pp = psum + (int64_t)ex * npsum;
+        for (int i = jx; i < npsum; i += P) ps += staged ? pp[i] : __ldcg(pp + i);
+    }
+    // P lanes of one warp per expert (P divides 32): a fixed xor tree
+    for (int o = P >> 1; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    if (ex < E && jx == 0) {
+        // group bases and the expert's total, in group order (integer sums); the
+        // group counts go back to zero
+        const int32_t* gh = ghist + (int64_t)ex * ng;
+        int32_t* gb = group_base + (int64_t)ex * ng;
         int run = 0;
-        for (int g0 = 0; g0 < ng; g0 += 32) {
-            const int g = g0 + lane;
-            const int v = g < ng ? (staged ? gh[g] : __ldcg(gh + g)) : 0;
-            const int incl = warp_inclusive_scan(v, lane);
-            if (g < ng) {
-                gb[g] = run + incl - v;
-                if (!staged) group_hist[(int64_t)e * ng + g] = 0;
-            }
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        double ps = 0.0;
-        if (npsum > 0) {
-            // fixed order: lane-strided partial sums, then a fixed xor tree
-            const double* pp = psum + (int64_t)e * npsum;
-            for (int i = lane; i < npsum; i += 32) ps += staged ? pp[i] : __ldcg(pp + i);
+        for (int g0 = 0; g0 < ng; g0 += 8) {
+            int v[8];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+            for (int u = 0; u < 8; ++u) v[u] = g0 + u < ng ? (staged ? gh[g0 + u] : __ldcg(gh + g0 + u)) : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (g0 + u < ng) {
+                    gb[g0 + u] = run;
+                    run += v[u];
+                    if (!staged) group_hist[(int64_t)ex * ng + g0 + u] = 0;
+                }
         }
-        if (lane == 0) {
-            sCount[e] = run;
-            sP[e] = ps;  // divided by the real-token count below
-            if (psum_total != nullptr) psum_total[e] = ps;
-        }
+        sCount[ex] = run;
+        sP[ex] = ps;  // divided by the real-token count below
+        if (psum_total != nullptr) psum_total[ex] = ps;
     }
     __syncthreads();
     if (warp == 0) {
