@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(kQThreads, 2) ffn_int8_kernel(const __grid_con
                 const uint8_t* st = smem + stage * kQStage;
                 // only the rows this pass holds (decode: one or two)
                 if (nr <= 1) consume_stage<TWO, 1>(st, w, lane, acc0, acc1);
-                else if (nr <= 2) consume_stage<TWO, 2>(st, w, lane, acc0, acc1);
+                else if (nr == 2) consume_stage<TWO, 2>(st, w, lane, acc0, acc1);
+                else if (nr == 3) consume_stage<TWO, 3>(st, w, lane, acc0, acc1);
                 else consume_stage<TWO, 4>(st, w, lane, acc0, acc1);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);
