@@ -45,6 +45,8 @@ constexpr int kQXTile = kQRows * kQKB * 2;  // 512 B of bf16 activations
 constexpr int kQStage = 2 * kQWTile + kQXTile;
 constexpr int kQRed = kQWarps * kQRows * kQCols * 2 * 4;  // partial sums of the 8 warps (32 KB)
 constexpr int kQSmem = kQStages * kQStage + kQRed + 256 + 128;
+static_assert(kQKB / kQWarps == 8, "a consumer warp takes 8 K rows: one 16-byte load of activations per row");
+static_assert(kQStage % 128 == 0, "stages stay 128-byte aligned");
 
 enum { Q_SWIGLU = 0, Q_GELU = 1, Q_PLAIN = 2, Q_PLAIN_BIAS = 3 };
 
@@ -135,7 +137,18 @@ __device__ __forceinline__ void consume_stage(const uint8_t* st, int w, int lane
     const uint32_t* w0 = reinterpret_cast<const uint32_t*>(st) + lane;
     const uint32_t* w1 = reinterpret_cast<const uint32_t*>(st + kQWTile) + lane;
     const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(st + 2 * kQWTile);
-#pragma unroll 4
+    // the warp's 8 activation values of each row, one 16-byte load per row (a bf16
+    // value widens to fp32 exactly by moving its bits to the upper half)
+    uint32_t xw[RT][4];
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + r * kQKB + w * (kQKB / kQWarps));
+        xw[r][0] = v.x;
+        xw[r][1] = v.y;
+        xw[r][2] = v.z;
+        xw[r][3] = v.w;
+    }
+#pragma unroll
     for (int i = 0; i < kQKB / kQWarps; ++i) {
         const int kk = w * (kQKB / kQWarps) + i;
         const uint32_t q0 = w0[kk * (kQCols / 4)];
@@ -145,7 +158,8 @@ __device__ __forceinline__ void consume_stage(const uint8_t* st, int w, int lane
         if (TWO) codes_to_pairs(q1, c1);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            const uint32_t xb = __float_as_uint(__bfloat162float(xs[r * kQKB + kk]));
+            const uint32_t h = xw[r][i >> 1];
+            const uint32_t xb = (i & 1) ? (h & 0xFFFF0000u) : (h << 16);
             const uint64_t xv = pack2(xb, xb);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {

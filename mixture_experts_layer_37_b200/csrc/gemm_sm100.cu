@@ -383,8 +383,11 @@ namespace {
 // runs a last tile of at most 128 rows as an M=128 pair tile).  The library's
 // choice, from same-machine measurements of both kernels on every benchmark
 // workload: the one-CTA kernel for the first GEMM (the pair was 1-7 % slower
-// there), and the pair for the second GEMM when an expert is expected to hold
-// at least 512 rows (its long-K tiles come in fewer, fuller waves).
+// there); for the second GEMM the pair when an expert is expected to hold at
+// least 512 rows and there are at most 16 experts (4096 and 8192 tokens over 8
+// experts: 110 vs 115 us and 1.58-1.61 vs 1.61-1.62 ms), else the one-CTA
+// kernel (32768 tokens over 32 experts: 1.17 vs 1.19-1.22 ms, where the pair
+// fetched its operands 1.45x over from DRAM).
 cudaError_t launch_one(int mode, bool pair, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int64_t rows_cap, cudaStream_t s) {
     if (p.gx != nullptr) {  // first GEMM with its rows gathered from the tokens (one-CTA kernel)
@@ -431,7 +434,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t s) {
     p1.k = a.k;
     // rows an expert is expected to receive (the routing itself stays on the device)
     const bool pair1 = a.gemm_kernel == MOE_GEMM_CTA_PAIR;
-    const bool pair2 = a.gemm_kernel == MOE_GEMM_CTA_PAIR || (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512);
+    const bool pair2 = a.gemm_kernel == MOE_GEMM_CTA_PAIR ||
+                       (a.gemm_kernel == MOE_GEMM_AUTO && a.rows_cap / a.E >= 512 && a.E <= 16);
     cudaError_t err = launch_one(swiglu ? MODE_SWIGLU : MODE_GELU, pair1, mA1, mB1, mB1u, p1, a.rows_cap, s);
     if (err != cudaSuccess) return err;
     if (a.between != nullptr && (err = record_mark(a.between, s)) != cudaSuccess) return err;
