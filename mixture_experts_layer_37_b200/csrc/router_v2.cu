@@ -551,15 +551,22 @@ __global__ void __launch_bounds__(kV2Threads, 1)
     }
     cluster_sync_all();  // no CTA leaves while a peer may still store into it or arrive on its barriers
     if (!a.fuse_scan) return;
-    // last CTA to finish runs the scan on everyone's statistics (its ring and weight slice as scratch)
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) sMisc[1] = (atomicAdd(a.counter, 1u) == gridDim.x - 1u) ? 1 : 0;
-    __syncthreads();
-    if (!sMisc[1]) return;
-    __threadfence();
+    // the scan on everyone's statistics (its ring and weight slice as scratch): with one cluster, rank 0
+    // runs it at once (the cluster barrier's release and acquire already ordered every CTA's results);
+    // otherwise the last CTA to finish
+    const bool one_cluster = gridDim.x == (unsigned)cs;
+    if (one_cluster) {
+        if (rank != 0) return;
+    } else {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) sMisc[1] = (atomicAdd(a.counter, 1u) == gridDim.x - 1u) ? 1 : 0;
+        __syncthreads();
+        if (!sMisc[1]) return;
+        __threadfence();
+    }
     scan_block(a.scan, sCount, sP, smem, nst * kStageBytes + va.slice_bytes);
-    if (threadIdx.x == 0) *a.counter = 0u;
+    if (threadIdx.x == 0 && !one_cluster) *a.counter = 0u;
 }
 
 struct V2Plan {

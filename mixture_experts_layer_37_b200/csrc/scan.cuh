@@ -115,21 +115,37 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
         if (psum_total != nullptr) psum_total[ex] = ps;
     }
     __syncthreads();
-    if (warp == 0) {
-        int32_t* __restrict__ counts = a.counts;
-        int32_t* __restrict__ offsets = a.offsets;
+    // two warps side by side: warp 0 the kept offsets, warp 1 (warp 0 in a one-warp block) the statistics,
+    // whose fp64 divisions are the longest chain left
+    const int stats_warp = nthreads > 32 ? 1 : 0;
+    if (warp == stats_warp && a.psum != nullptr) {
         float* __restrict__ fo = a.f;
         float* __restrict__ po = a.p;
         float* __restrict__ lo = a.l_aux;
+        // the real-token count is final: every producer added to it before the scan started
+        const int64_t t_real = real_counter != nullptr ? (int64_t)__ldcg(real_counter) : T;
+        // statistics in a fixed order: lane-strided partial sums, then a fixed xor tree
+        double l = 0.0;
+        for (int e = lane; e < E; e += 32) {
+            const double f = t_real > 0 ? (double)sCount[e] / ((double)t_real * k) : 0.0;
+            const double pe = t_real > 0 ? sP[e] / (double)t_real : 0.0;
+            if (fo) fo[e] = (float)f;
+            if (po) po[e] = (float)pe;
+            l += f * pe;
+        }
+        double tot = l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        if (lane == 0 && lo) lo[0] = (float)((double)a.alpha * E * tot);
+    }
+    if (warp == 0) {
+        int32_t* __restrict__ counts = a.counts;
+        int32_t* __restrict__ offsets = a.offsets;
         int32_t* __restrict__ t_real_out = a.t_real_out;
         int32_t* __restrict__ shared_off = a.shared_off;
-        const bool stats = a.psum != nullptr;
-        const float alpha = a.alpha;
         // real tokens: every token, or the router's count of unmasked tokens
         int64_t t_real = T;
         if (real_counter != nullptr) t_real = __ldcg(real_counter);
-        __syncwarp();
-        if (lane == 0 && real_counter != nullptr) *real_counter = 0;
         if (lane == 0 && t_real_out != nullptr) t_real_out[0] = (int32_t)t_real;
         if (lane == 0 && shared_off != nullptr) {
             shared_off[0] = 0;
@@ -148,22 +164,10 @@ __device__ __forceinline__ void scan_block(const ScanArgs& a, int* sCount, doubl
             run += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) offsets[E] = run;
-        if (stats) {
-            // statistics in a fixed order: lane-strided partial sums, then a fixed xor tree
-            double l = 0.0;
-            for (int e = lane; e < E; e += 32) {
-                const double f = t_real > 0 ? (double)sCount[e] / ((double)t_real * k) : 0.0;
-                const double pe = t_real > 0 ? sP[e] / (double)t_real : 0.0;
-                if (fo) fo[e] = (float)f;
-                if (po) po[e] = (float)pe;
-                l += f * pe;
-            }
-            double tot = l;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-            if (lane == 0 && lo) lo[0] = (float)((double)alpha * E * tot);
-        }
     }
+    // the real-token counter goes back to zero once both warps have read it
+    __syncthreads();
+    if (tid == 0 && real_counter != nullptr) *real_counter = 0;
 }
 
 // The rank base of chunk `chunk` for expert e: its group's base plus the
