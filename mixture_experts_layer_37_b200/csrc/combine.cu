@@ -23,6 +23,8 @@ namespace {
 // this step's all-to-all, fused with the weighted sum.
 template <bool BF16, bool EP, int U>  // U: 16-byte vectors per lane per expert row (x2 rows in flight)
 __global__ void __launch_bounds__(256, 8 / U) combine_kernel(CombineArgs a) {
+    griddep_wait();  // the expert rows of the launches before
+    griddep_launch_dependents();
     constexpr int VEC = BF16 ? 8 : 4;  // elements per 16-byte vector
     const int warps_per_cta = blockDim.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -215,16 +217,13 @@ __global__ void selftest_wait_kernel(DevStatus st) {
 }
 
 template <int U>
-void launch_combine_u(const CombineArgs& a, bool bf16, int64_t blocks, cudaStream_t s) {
+cudaError_t launch_combine_u(const CombineArgs& a, bool bf16, int64_t blocks, cudaStream_t s) {
     const bool ep = a.e_per_rank > 0;
-    if (bf16 && ep)
-        combine_kernel<true, true, U><<<(unsigned)blocks, 256, 0, s>>>(a);
-    else if (bf16)
-        combine_kernel<true, false, U><<<(unsigned)blocks, 256, 0, s>>>(a);
-    else if (ep)
-        combine_kernel<false, true, U><<<(unsigned)blocks, 256, 0, s>>>(a);
-    else
-        combine_kernel<false, false, U><<<(unsigned)blocks, 256, 0, s>>>(a);
+    const dim3 grid((unsigned)blocks), block(256);
+    if (bf16 && ep) return launch_kernel(combine_kernel<true, true, U>, grid, block, 0, s, a);
+    if (bf16) return launch_kernel(combine_kernel<true, false, U>, grid, block, 0, s, a);
+    if (ep) return launch_kernel(combine_kernel<false, true, U>, grid, block, 0, s, a);
+    return launch_kernel(combine_kernel<false, false, U>, grid, block, 0, s, a);
 }
 
 }  // namespace
@@ -234,8 +233,7 @@ void launch_combine_u(const CombineArgs& a, bool bf16, int64_t blocks, cudaStrea
 // vectors per lane, were measured slower: half the warps fit per SM.)
 cudaError_t launch_combine(const CombineArgs& a, bool bf16, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
-    launch_combine_u<4>(a, bf16, min64((a.T + 7) / 8, (int64_t)sm_count() * 8), s);
-    return cudaGetLastError();
+    return launch_combine_u<4>(a, bf16, min64((a.T + 7) / 8, (int64_t)sm_count() * 8), s);
 }
 
 

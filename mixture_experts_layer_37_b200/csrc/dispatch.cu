@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScanArgs a) {
 __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a, int nsplit) {
     __shared__ int sWarpBase[kScatterWarps][kMaxExperts];
     __shared__ uint4* sDst[kScatterThreads];
+    griddep_wait();  // the routing of the launch before
+    griddep_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, k = a.k;
     const int chunk = blockIdx.x / nsplit, part = blockIdx.x - chunk * nsplit;
@@ -313,8 +315,7 @@ cudaError_t launch_dispatch_scatter(const ScatterArgs& a, cudaStream_t s) {
     int nsplit = 1;
     const bool copies = a.x_perm != nullptr || a.e_per_rank > 0;
     while (copies && nsplit < 4 && (int64_t)a.nchunk * nsplit < 2 * (int64_t)sm_count()) nsplit *= 2;
-    scatter_kernel<<<(unsigned)(a.nchunk * nsplit), kScatterThreads, 0, s>>>(a, nsplit);
-    return cudaGetLastError();
+    return launch_kernel(scatter_kernel, dim3((unsigned)(a.nchunk * nsplit)), dim3(kScatterThreads), 0, s, a, nsplit);
 }
 
 }  // namespace moe

@@ -184,6 +184,8 @@ __global__ void __launch_bounds__(kQThreads, 2) ffn_int8_kernel(const __grid_con
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kQStage + kQRed);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQStages);
+    griddep_wait();  // the rows and offsets of the launches before
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.y;
     const int row_begin = p.offsets[e], row_end = p.offsets[e + 1];
@@ -321,8 +323,7 @@ cudaError_t launch_q(const CUtensorMap& q0, const CUtensorMap& q1, const CUtenso
     const cudaError_t err = ensure_smem_attr(attr, ffn_int8_kernel<MODE>, kQSmem);
     if (err != cudaSuccess) return err;
     dim3 grid((p.N + kQCols - 1) / kQCols, E);
-    ffn_int8_kernel<MODE><<<grid, kQThreads, kQSmem, s>>>(q0, q1, a, p);
-    return cudaGetLastError();
+    return launch_kernel(ffn_int8_kernel<MODE>, grid, dim3(kQThreads), kQSmem, s, q0, q1, a, p);
 }
 
 }  // namespace

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtParams p) {
     __shared__ int mt_prefix[kMaxExperts + 1];
     __shared__ float As[TK][TM + 4];
     __shared__ float Bs[2][TK][TN];
+    griddep_wait();  // the rows and offsets of the launches before
+    griddep_launch_dependents();
     if (threadIdx.x == 0) {
         int acc = 0;
         mt_prefix[0] = 0;
@@ -110,7 +112,8 @@ template <int MODE>
 cudaError_t launch_simt(const SimtParams& p, int64_t rows_cap, cudaStream_t s) {
     const int64_t tiles = (rows_cap / TM + p.E) * (int64_t)p.n_tiles;
     if (tiles <= 0) return cudaSuccess;
-    simt_gemm_kernel<MODE><<<(unsigned)tiles, 256, 0, s>>>(p);
+    const cudaError_t err = launch_kernel(simt_gemm_kernel<MODE>, dim3((unsigned)tiles), dim3(256), 0, s, p);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 

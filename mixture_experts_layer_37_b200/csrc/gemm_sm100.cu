@@ -95,6 +95,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    // the prologue above overlaps the launch before; from here on its results are read
+    griddep_wait();
+    griddep_launch_dependents();
     if (threadIdx.x == 64) build_tile_table(p, BM, mt_prefix, s_off);
     tc_fence_before();
     __syncthreads();
@@ -339,8 +342,7 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     const int64_t tiles_upper = (rows_cap / BM + p.E) * (int64_t)p.n_tiles;
     const int grid = (int)min64(tiles_upper, (int64_t)sm_count());
     if (grid <= 0) return cudaSuccess;
-    grouped_gemm_kernel<MODE, GATHER><<<grid, kThreads, kSmemBytes, s>>>(a, b0, b1, p);
-    return cudaGetLastError();
+    return launch_kernel(grouped_gemm_kernel<MODE, GATHER>, dim3(grid), dim3(kThreads), kSmemBytes, s, a, b0, b1, p);
 }
 
 }  // namespace

@@ -169,6 +169,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_alloc_pair(tmem_slot, kTmemCols);
         tmem_relinquish_pair();
     }
+    // the prologue above overlaps the launch before; from here on its results are read
+    griddep_wait();
+    griddep_launch_dependents();
     if (threadIdx.x == 64) build_tile_table(p, BMP, mt_prefix, s_off);
     tc_fence_before();
     __syncthreads();
@@ -358,8 +361,7 @@ cudaError_t launch_pair_mode(const CUtensorMap& a, const CUtensorMap& b0, const 
     const int64_t tiles_upper = (rows_cap / BMP + p.E) * (int64_t)p.n_tiles;
     const int pairs = (int)min64(tiles_upper, (int64_t)pairs_cap);
     if (pairs <= 0) return cudaSuccess;
-    grouped_gemm_pair_kernel<MODE><<<2 * pairs, kThreads, kSmemP, s>>>(a, b0, b1, p);
-    return cudaGetLastError();
+    return launch_kernel(grouped_gemm_pair_kernel<MODE>, dim3(2 * pairs), dim3(kThreads), kSmemP, s, a, b0, b1, p);
 }
 
 }  // namespace

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <atomic>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -225,6 +226,38 @@ cudaError_t launch_quantize_int8(const void* w, bool bf16, int64_t E, int64_t K,
 cudaError_t launch_selftest_wait(DevStatus st, cudaStream_t s);
 
 int sm_count();
+
+// Programmatic dependent launch inside one forward.  While a PdlScope lives on
+// this host thread, launch_kernel starts kernels with programmatic stream
+// serialization: a kernel's launch and prologue overlap the tail of the kernel
+// before it on the stream.  Every kernel launched that way executes
+// griddep_wait() before it reads anything an earlier kernel wrote (for a
+// kernel launched without the attribute that wait returns at once).
+bool pdl_enabled();
+struct PdlScope {
+    PdlScope();
+    ~PdlScope();
+    PdlScope(const PdlScope&) = delete;
+    PdlScope& operator=(const PdlScope&) = delete;
+    bool prev;
+};
+template <class... KArgs, class... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (pdl_enabled()) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Raises a kernel's dynamic shared-memory limit once per device.  Safe from
 // several host threads: concurrent first calls may both set it (idempotent).

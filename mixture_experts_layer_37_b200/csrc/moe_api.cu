@@ -24,6 +24,13 @@ int sm_count() {
     return n;
 }
 
+namespace {
+thread_local bool t_pdl = false;
+}
+bool pdl_enabled() { return t_pdl; }
+PdlScope::PdlScope() : prev(t_pdl) { t_pdl = true; }
+PdlScope::~PdlScope() { t_pdl = prev; }
+
 }  // namespace moe
 
 namespace {
@@ -597,6 +604,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const moe_weights_t* w
     if (!mark()) return MOE_ERR_CUDA;
     const bool gather = gathers(cfg);
     const bool weighted = weights_in_epilogue(cfg);
+    // the launches after the router overlap each predecessor's tail (programmatic dependent launch)
+    const PdlScope pdl;
     {
         const NvtxRange r("moe_forward/scatter");
         st = run_scatter(cfg, x, o->topk_idx, o->offsets, o->slot, o->src_assign, gather ? nullptr : x_perm, ws, pl,
