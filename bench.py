@@ -300,30 +300,15 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
     torch.cuda.synchronize()
     eager_ms = float(sum(ev[0].elapsed_time(ev[nl]) for ev in eager))
 
-    # the timed region: K steps of the user's call (moe_forward) captured into one graph, an event
-    # on each side of every step; the L2 clearing between steps lies outside them
-    step_ev = [make_events(2) for _ in range(steps)]
+    # the timed region: K steps captured into one graph
+    step_ev = [make_events(nl + 1) for _ in range(steps)]
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for i in range(steps):
             clear_l2()
-            step_ev[i][0].record(stream)
-            M.moe_forward(cfg, weights, x, layer.outputs, layer.ws, token_mask=tmask)
-            step_ev[i][1].record(stream)
+            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, step_ev[i], token_mask=tmask)
     graph.replay()  # upload and warm the graph
-    torch.cuda.synchronize()
-    layer.check()
-    # the stage breakdown: the same steps with an event between every two launches (the events
-    # keep each launch from overlapping the one before, so these steps run a little longer)
-    stage_ev = [make_events(nl + 1) for _ in range(steps)]
-    torch.cuda.synchronize()
-    sgraph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(sgraph):
-        for i in range(steps):
-            clear_l2()
-            M.moe_forward_profiled(cfg, weights, x, layer.outputs, layer.ws, stage_ev[i], token_mask=tmask)
-    sgraph.replay()
     torch.cuda.synchronize()
     layer.check()
     dev_id = str(torch.cuda.get_device_properties(local).uuid) if hasattr(torch.cuda.get_device_properties(local), "uuid") else str(local)
@@ -341,10 +326,8 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
     clocks = sampler.stop()
     layer.check()
 
-    sgraph.replay()  # the stage breakdown, warm
-    torch.cuda.synchronize()
-    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in stage_ev])
-    step_ms = np.array([ev[0].elapsed_time(ev[1]) for ev in step_ev])
+    stage_ms = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(nl)] for ev in step_ev])
+    step_ms = np.array([ev[0].elapsed_time(ev[nl]) for ev in step_ev])
     total_ms = float(step_ms.sum())
     if world > 1:
         t = torch.tensor([total_ms, eager_ms], dtype=torch.float64, device="cuda")
@@ -501,13 +484,12 @@ def bench_workload(a, name: str, steps: int, warmup: int, cpu_seconds: float, wo
                    "act": wl.act, "capacity_factor": wl.capacity_factor, "rows_dispatched": R,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
-                   "launch": "timed steps (moe_forward) replayed from one captured CUDA graph; stages from a "
-                             "second graph of the same steps with an event between launches",
+                   "launch": "timed steps replayed from one captured CUDA graph",
                    "router_kernel": a.router_kernel, "gemm_kernel": a.gemm_kernel, "dispatch": a.dispatch},
         "roofline": roofline, "forward_roofline": forward_roofline, "stages": stages, "e2e": e2e, "gpu_launches": nl * steps,
         "clocks": clocks, "cpu_baseline": cpu,
     }
-    del layer, weights, x, flush, evict, graph, sgraph
+    del layer, weights, x, flush, evict, graph
     torch.cuda.empty_cache()
     return line
 
