@@ -326,7 +326,11 @@ moe_status_t moe_aux_stats(const moe_config_t* cfg, const int32_t* counts, const
  *     accumulated in fp32 (routed terms first, then shared experts in order)
  *     and rounded once.
  *   cfg->weighting: whether w[t,j] y(t,j) is formed in the second GEMM's
- *     epilogue (rounded there) or in the combine (moe_weighting_t). */
+ *     epilogue (rounded there) or in the combine (moe_weighting_t).
+ * Every launch after the router uses programmatic dependent launch: it may
+ * start while the kernel before it finishes and waits on the device before
+ * reading that kernel's results (no effect on results; the router itself is
+ * launched plainly, so consecutive forwards on a stream never overlap). */
 moe_status_t moe_forward(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
                          const float* logits_in, const uint8_t* token_mask, moe_outputs_t* outputs, void* ws,
                          size_t ws_bytes, cudaStream_t stream);
